@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark over a paged KV cache (one JSON line on rank 0).
+
+A step is one call of the library's decode entry point (device-side split
+planning, the decode kernel and the LSE-combine kernel) over one batch of the
+synthetic workload.  Default workload: GTA decode, batch 32, q_len 1, h_q 32,
+8 tied KV groups, d_h 128, shared RoPE slice 64, contexts uniform in
+[1024, 8192], page size 64, shuffled block table.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gta|gqa|mla|gla2] [--qlen L]
+  python bench.py --impl reference ...   # the fp64 CPU oracle timed on this host
+
+Multi-GPU: the path has no exchange step (sequences are independent), so N GPUs
+run N independent replicas of the step (weak scaling, no collective on the data
+path); the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_paged_b200 import accounting, workload as wl  # noqa: E402
+
+METRIC = "decode-attention µs/step and KV-cache GB/s as % of B200 HBM peak (1 GPU)"
+UNIT = "us/step"
+FALLBACK_HBM_GBS, FALLBACK_TFLOPS = 6650.0, 1590.0
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
+KERNEL_SOURCES = {"group": ["kv_cache_paged_b200/csrc/group_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"],
+                  "latent": ["kv_cache_paged_b200/csrc/latent_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"]}
+
+
+def describe(inp):
+    sl = inp.seqlens
+    if inp.variant == "gla":
+        kind = "MLA" if inp.h_kv == 1 else f"GLA-{inp.h_kv}"
+        shape = f"h_q {inp.h_q}, h_c {inp.h_kv}, d_c {inp.d}, d_r {inp.d_r}"
+    elif inp.variant == "gta":
+        kind, shape = "GTA", f"h_q {inp.h_q}, h_kv {inp.h_kv}, d_h {inp.d}, d_r {inp.d_r}"
+    else:
+        kind, shape = "GQA", f"h_q {inp.h_q}, h_kv {inp.h_kv}, d {inp.d}"
+    return (f"{kind} paged decode: B {inp.B}, q_len {inp.L}, {shape}, page {inp.page_size}, "
+            f"contexts {int(sl.min())}..{int(sl.max())} (mean {float(sl.mean()):.0f})")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_TFLOPS, "fallback"
+
+
+def kernel_hash(kind):
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kind]:
+        p = os.path.join(ROOT, rel)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kind, workload, qlen):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(f"{workload}_L{qlen}")
+        if e and e.get("kernel_sha") == kernel_hash(kind):
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples for one GPU while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.rows = []
+        self.proc = None
+        self.t_on = self.t_off = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.th = threading.Thread(target=self._read, daemon=True)
+        self.th.start()
+        time.sleep(0.5)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), line.strip()))
+
+    def mark_on(self):
+        self.t_on = time.time()
+
+    def mark_off(self):
+        self.t_off = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [r for t, r in self.rows if self.t_on is not None and self.t_on - 0.1 <= t <= self.t_off + 0.15]
+        if not rows:
+            rows = [r for _, r in self.rows]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+def oracle_sample(inp, budget_s):
+    """Time the fp64 oracle on a prefix of the batch sized to about budget_s seconds of CPU work.
+    Returns (seconds, fraction of the step's work, threads, sequences)."""
+    from oracle import oracle as orc
+    work = np.maximum(inp.seqlens.astype(np.float64), 0)
+    total = work.sum()
+    t0 = time.perf_counter()
+    _, _, threads = orc.decode_inputs(inp, b_list=np.array([0], np.int32))
+    t1 = time.perf_counter() - t0
+    per_tok = t1 / max(work[0], 1)
+    n, acc = 0, 0.0
+    while n < inp.B and (acc + work[n]) * per_tok <= budget_s:
+        acc += work[n]
+        n += 1
+    n = max(n, 1)
+    bl = np.arange(n, dtype=np.int32)
+    t0 = time.perf_counter()
+    _, _, threads = orc.decode_inputs(inp, b_list=bl)
+    dt = time.perf_counter() - t0
+    return dt, float(work[:n].sum() / total), threads, n
+
+
+def run_reference(args, inp, cfg, rank):
+    """The reference arm: the fp64 CPU oracle, timed as it stands on this host."""
+    if rank != 0:
+        return
+    K, W = args.steps, args.warmup
+    budget = max(0.02, min(2.0, 150.0 / max(1, K + W)))
+    for _ in range(W):
+        oracle_sample(inp, budget)
+    per_step = []
+    frac = threads = n = None
+    for _ in range(K):
+        dt, frac, threads, n = oracle_sample(inp, budget)
+        per_step.append(dt / frac * 1e6)
+    v = float(statistics.mean(per_step))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": K,
+            "warmup": W, "ms_per_step": v / 1e3, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"first {n} of {inp.B} sequences per step ({frac:.3f} of the step's "
+                                       f"work), time scaled to the whole step"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="kvd", choices=["kvd", "reference"])
+    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny"])
+    ap.add_argument("--qlen", type=int, default=1)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+
+    inp = wl.make_workload(args.workload, L=args.qlen)
+    nbytes, flops, kvb = accounting.of_inputs(inp)
+    cfg = {"workload": describe(inp), "global_batch": inp.B * world, "seq_len": int(inp.seqlens.max()),
+           "q_len": inp.L, "seed": wl.SEEDS[args.workload], "parallelism": f"replicas{world}",
+           "l2": "flushed before every timed step (256 MiB write); the KV stream is also larger than L2",
+           "kv_bytes_per_step": int(kvb), "algorithmic_bytes_per_step": int(nbytes),
+           "flops_per_step": int(flops)}
+
+    if args.impl == "reference":
+        run_reference(args, inp, cfg, rank)
+        return
+
+    import torch
+    from kv_cache_paged_b200 import binding
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    caches = {k: bf(v).to(dev) for k, v in inp.caches.items()}
+    q_h = bf(inp.q).pin_memory()
+    bt_h = torch.from_numpy(inp.block_table).pin_memory()
+    sl_h = torch.from_numpy(inp.seqlens).pin_memory()
+    q, bt, sl = q_h.to(dev), bt_h.to(dev), sl_h.to(dev)
+    d_v = inp.d
+    out = torch.empty((inp.B, inp.L, inp.h_q, d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((inp.B, inp.L, inp.h_q), dtype=torch.float32, device=dev)
+    out_h = torch.empty_like(out, device="cpu").pin_memory()
+    lse_h = torch.empty_like(lse, device="cpu").pin_memory()
+    ws = torch.zeros(1 << 30 if inp.variant == "gla" else 1 << 26, dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    names = {"gqa": ("k_cache", "v_cache"), "gta": ("tied_cache", "rope_cache"),
+             "gla": ("latent_cache", "rope_cache")}[inp.variant]
+    fn = {"gqa": binding.gqa_decode, "gta": binding.gta_decode, "gla": binding.gla_decode}[inp.variant]
+    c0, c1 = caches[names[0]], caches[names[1]]
+    launches_per_step = 2  # decode kernel (planning fused in) + LSE combine
+
+    def step(qq, btt, sll):
+        fn(qq, c0, c1, btt, sll, inp.scale, out=out, lse=lse, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            step(q, bt, sl)
+    err = binding.read_device_error(ws, stream)
+    if err:
+        raise SystemExit(f"device error flags after warm-up: {err}")
+
+    gpu_index = torch.cuda.get_device_properties(dev).uuid if hasattr(torch.cuda.get_device_properties(dev), "uuid") else local
+    sampler = ClockSampler(f"GPU-{gpu_index}" if not isinstance(gpu_index, int) else gpu_index)
+    sampler.start()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    with torch.cuda.stream(stream):
+        for k in range(K):          # create the kernel events (torch creates them lazily on record)
+            ev[k][1].record(stream)
+            ev[k][2].record(stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.mark_on()
+    t_wall = time.perf_counter()
+    with torch.cuda.stream(stream):
+        for k in range(K):
+            flush.fill_(k & 0xFF)
+            e0, kb, ka, e1 = ev[k]
+            binding.profile_events(kb, ka)
+            e0.record(stream)
+            step(q, bt, sl)
+            e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t_wall = time.perf_counter() - t_wall
+    sampler.mark_off()
+    binding.profile_events(None, None)
+    step_ms = [ev[k][0].elapsed_time(ev[k][3]) for k in range(K)]
+    kern_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    clocks = sampler.stop()
+
+    # end to end through the public API with host buffers: H2D of the step's inputs
+    # (q, seqlens, block table) from pinned memory, the call, D2H of out and lse.
+    KE = max(1, min(args.e2e_steps, K))
+    ee = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(KE)]
+    with torch.cuda.stream(stream):
+        for k in range(KE):
+            flush.fill_(k & 0xFF)
+            ee[k][0].record(stream)
+            q.copy_(q_h, non_blocking=True)
+            sl.copy_(sl_h, non_blocking=True)
+            bt.copy_(bt_h, non_blocking=True)
+            step(q, bt, sl)
+            out_h.copy_(out, non_blocking=True)
+            lse_h.copy_(lse, non_blocking=True)
+            ee[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = [ee[k][0].elapsed_time(ee[k][1]) for k in range(KE)]
+    err = binding.read_device_error(ws, stream)
+    if err:
+        raise SystemExit(f"device error flags after timing: {err}")
+
+    t_step = statistics.mean(step_ms)
+    t_kern = statistics.mean(kern_ms)
+    t_e2e = statistics.mean(e2e_ms)
+    if pg is not None:
+        v = torch.tensor([t_step, t_kern, t_e2e], dtype=torch.float64, device=dev)
+        pg.all_reduce(v, op=pg.ReduceOp.MAX)
+        t_step, t_kern, t_e2e = (float(x) for x in v.tolist())
+
+    hbm, tfl, peak_src = load_peaks()
+    variant_kind = "latent" if inp.variant == "gla" else "group"
+    tensor_bound = flops / (tfl * 1e12) > nbytes / (hbm * 1e9)
+    if tensor_bound:
+        achieved = flops / (t_kern * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tfl, "unit": "TFLOP/s", "frac": achieved / tfl}
+    else:
+        achieved = nbytes / (t_kern * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm}
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    roof["kernel"] = "group_decode_kernel" if variant_kind == "group" else "latent_decode_kernel"
+    roof["kernel_us"] = t_kern * 1e3
+    roof["traffic"] = committed_traffic(variant_kind, args.workload, inp.L)
+    roof["roofline_us"] = accounting.roofline_us(nbytes, flops, hbm, tfl)
+
+    kv_gbs = kvb / (t_step * 1e-3) / 1e9
+    line = {"metric": METRIC, "value": t_step * 1e3, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "kv_gbs": kv_gbs * world, "kv_gbs_per_gpu": kv_gbs, "kv_frac_of_hbm_peak": kv_gbs / hbm,
+            "step_us_p10_p50_p90": [float(np.percentile(step_ms, p) * 1e3) for p in (10, 50, 90)],
+            "roofline_frac_of_step": roof["roofline_us"] / (t_step * 1e3),
+            "roofline": roof,
+            "e2e": {"value": t_e2e * 1e3, "unit": UNIT,
+                    "h2d_bytes_per_step": int(q.numel() * 2 + sl.numel() * 4 + bt.numel() * 4),
+                    "d2h_bytes_per_step": int(out.numel() * 2 + lse.numel() * 4)},
+            "gpu_launches": K * launches_per_step, "timed_region_wall_s": t_wall,
+            "clocks": clocks}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, frac, threads, n = oracle_sample(inp, args.cpu_budget)
+        line["cpu_baseline"] = {"value": dt / frac * 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"first {n} of {inp.B} sequences ({frac:.3f} of the step's work) "
+                                          f"in {dt:.1f} s, scaled to the whole step"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

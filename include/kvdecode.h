@@ -1,0 +1,204 @@
+/*
+ * kvdecode — decode-phase attention over a paged KV cache on NVIDIA B200 (sm_100a).
+ *
+ * Variants, as defined in "Hardware-Efficient Attention for Fast Decoding"
+ * (Zadouri, Strauss, Dao; section 3 "Methodology", Figure 2 caption):
+ *   GQA  query heads split into h_kv groups; each group reads its own K and V
+ *        head (m_kv = 2).  MQA (h_kv = 1) and MHA (h_kv = h_q) are special cases.
+ *   GTA  grouped-tied attention: one tied state per group is the value (all d_h
+ *        dims) and its first d_h - d_r dims are the non-RoPE half of the key;
+ *        the RoPE half of the key is one d_r-wide slice per token shared by all
+ *        heads (m_kv = 1).
+ *   GLA  grouped latent attention in absorbed form: h_c latent heads of width
+ *        d_c plus one shared d_r-wide RoPE key; query head h attends latent head
+ *        h / (h_q / h_c) with key = [latent ++ rope] and value = latent.  MLA is
+ *        the h_c = 1 case.
+ *
+ * For sequence b with T_b = seqlens[b] cached tokens (the L new query tokens
+ * are the last L of them), query row i in [0, L) and head h:
+ *   visible tokens t <= T_b - L + i;  s_t = scale * <q, k_t>;
+ *   lse = ln sum_t exp(s_t);  out = sum_t exp(s_t - lse) v_t.
+ * A row that sees no token gets out = 0 and lse = -inf.
+ *
+ * Memory (all pointers are DEVICE pointers owned by the caller; the library
+ * never allocates, frees or keeps them after the call returns):
+ *   q            bf16 [B, L, h_q, d_qk] contiguous
+ *                  GQA d_qk = d; GTA d_qk = d_h laid out [q_nope (d_h - d_r) ++ q_rope (d_r)];
+ *                  GLA d_qk = d_c + d_r laid out [q_latent (d_c) ++ q_rope (d_r)]
+ *   caches       bf16, page-major: [num_pages, page_size, heads, dim] contiguous
+ *                  GQA k_cache, v_cache [P, S, h_kv, d]
+ *                  GTA tied_cache [P, S, h_kv, d_h], rope_cache [P, S, d_r]
+ *                  GLA latent_cache [P, S, h_c, d_c], rope_cache [P, S, d_r]
+ *                RoPE is applied when tokens are written (rotated keys are
+ *                stored, q arrives rotated); decode does no rotation.
+ *   block_table  int32 [B, max_pages]: physical page of logical page i of b.
+ *                Entries at or past ceil(T_b / page_size) are never read.
+ *   seqlens      int32 [B], 0 <= T_b <= max_pages * page_size, and T_b >= L
+ *                when T_b > 0.
+ *   out          bf16 [B, L, h_q, d_v] (d_v = d, d_h or d_c), round to nearest even
+ *   lse          fp32 [B, L, h_q], natural log of the softmax denominator of the
+ *                scaled scores
+ *   workspace    device scratch of at least kvd_*_workspace_size() bytes, 256-byte
+ *                aligned, ZEROED ONCE before its first use (cudaMemset).  It holds
+ *                the split-KV partials and a sticky device error word; calls
+ *                that overlap on the GPU must not share one workspace.
+ * All base pointers must be 16-byte aligned (TMA).
+ *
+ * Execution: every entry point is asynchronous on `stream`; there is no host
+ * synchronisation and no allocation, so a call can be captured in a CUDA graph.
+ * Split planning runs on the device from seqlens: the (sequence, 16-token tile)
+ * stream is cut into `num_parts` equal contiguous parts (0 = one per SM, or per
+ * SM pair for the latent kernel), each processed by one CTA; sequences cut into
+ * several parts are merged by an LSE-combine kernel.
+ *
+ * Errors: functions return KVD_OK (0) or a negative KVD_ERR_* code and do not
+ * launch anything on a host-side validation error.  Faults detected on the
+ * device (a block-table entry outside [0, num_pages), an invalid seqlen, a
+ * bounded wait that ran out) never trap: the kernel records a flag in the
+ * workspace's error word, substitutes a safe value (page 0, a clamped length)
+ * or stops early, and kvd_read_device_error() reports it.
+ */
+#ifndef KVDECODE_H
+#define KVDECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kvd_stream_t; /* same handle as cudaStream_t; NULL = legacy default stream */
+
+enum {
+    KVD_OK = 0,
+    KVD_ERR_INVALID_ARG = -1,        /* null/misaligned pointer, inconsistent sizes */
+    KVD_ERR_UNSUPPORTED_SHAPE = -2,  /* head dims / page size outside the compiled set */
+    KVD_ERR_WORKSPACE_TOO_SMALL = -3,
+    KVD_ERR_CUDA = -4,               /* a CUDA runtime call or launch failed */
+    KVD_ERR_DEVICE = -5              /* kvd_read_device_error found flags set */
+};
+
+/* Device error-word bits reported by kvd_read_device_error(). */
+enum {
+    KVD_DEVERR_TIMEOUT = 1u,     /* a bounded pipeline wait ran out; output incomplete */
+    KVD_DEVERR_BAD_PAGE = 2u,    /* block_table entry outside [0, num_pages); page 0 was read instead */
+    KVD_DEVERR_BAD_SEQLEN = 4u   /* seqlens[b] < 0, > max_pages*page_size, or 0 < T_b < L; clamped */
+};
+
+/*
+ * GQA (and MQA/MHA).  d in {64, 128}; h_q % h_kv == 0; (h_q / h_kv) * L <= 32;
+ * page_size a multiple of 16.
+ */
+typedef struct {
+    const void *q;            /* bf16 [B, L, h_q, d] */
+    const void *k_cache;      /* bf16 [num_pages, page_size, h_kv, d] */
+    const void *v_cache;      /* bf16 [num_pages, page_size, h_kv, d] */
+    const int32_t *block_table;
+    const int32_t *seqlens;
+    void *out;                /* bf16 [B, L, h_q, d] */
+    float *lse;               /* fp32 [B, L, h_q] */
+    int32_t B, L, h_q, h_kv, d, page_size, num_pages, max_pages;
+    float scale;              /* softmax scale applied to q.k */
+    int32_t num_parts;        /* 0 = auto */
+} kvd_gqa_params;
+
+/*
+ * GTA.  d_h in {64, 128}, d_r in {32, 64}, d_r <= d_h, (d_h - d_r) % 16 == 0;
+ * other limits as GQA.
+ */
+typedef struct {
+    const void *q;            /* bf16 [B, L, h_q, d_h] = [nope ++ rope] */
+    const void *tied_cache;   /* bf16 [num_pages, page_size, h_kv, d_h] */
+    const void *rope_cache;   /* bf16 [num_pages, page_size, d_r] */
+    const int32_t *block_table;
+    const int32_t *seqlens;
+    void *out;                /* bf16 [B, L, h_q, d_h] */
+    float *lse;               /* fp32 [B, L, h_q] */
+    int32_t B, L, h_q, h_kv, d_h, d_r, page_size, num_pages, max_pages;
+    float scale;
+    int32_t num_parts;
+} kvd_gta_params;
+
+/*
+ * GLA / MLA (absorbed).  d_c in {256, 512}, d_r == 64, h_q % h_c == 0,
+ * (h_q / h_c) * L <= 256, page_size a multiple of 64.
+ */
+typedef struct {
+    const void *q;            /* bf16 [B, L, h_q, d_c + d_r] = [latent ++ rope] */
+    const void *latent_cache; /* bf16 [num_pages, page_size, h_c, d_c] */
+    const void *rope_cache;   /* bf16 [num_pages, page_size, d_r] */
+    const int32_t *block_table;
+    const int32_t *seqlens;
+    void *out;                /* bf16 [B, L, h_q, d_c] */
+    float *lse;               /* fp32 [B, L, h_q] */
+    int32_t B, L, h_q, h_c, d_c, d_r, page_size, num_pages, max_pages;
+    float scale;
+    int32_t num_parts;
+} kvd_gla_params;
+
+/* Bytes of workspace the matching decode call needs (0 on invalid params). */
+size_t kvd_gqa_workspace_size(const kvd_gqa_params *p);
+size_t kvd_gta_workspace_size(const kvd_gta_params *p);
+size_t kvd_gla_workspace_size(const kvd_gla_params *p);
+
+/* Decode entry points: plan, decode and combine kernels on `stream`. */
+int kvd_gqa_decode(const kvd_gqa_params *p, void *workspace, size_t workspace_bytes, kvd_stream_t stream);
+int kvd_gta_decode(const kvd_gta_params *p, void *workspace, size_t workspace_bytes, kvd_stream_t stream);
+int kvd_gla_decode(const kvd_gla_params *p, void *workspace, size_t workspace_bytes, kvd_stream_t stream);
+
+/*
+ * Split plan for inspection and tests.  Cuts the (sequence, tile) stream of
+ * seqlens[B] (device pointer) with `tile` tokens per tile into num_parts parts
+ * exactly as the decode kernels do and writes, for part c, up to `cap` records
+ * of 6 int32 {b, tile_begin, tile_end, split_index, num_splits, slot} at
+ * segments[c * cap * 6 ...] and the record count at counts[c] (device
+ * pointers).  A count above `cap` means records were dropped.
+ */
+int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_tokens, int32_t num_parts,
+             int32_t *segments, int32_t *counts, int32_t cap, kvd_stream_t stream);
+
+/* The same plan computed on the host from host memory; returns KVD_OK. */
+int kvd_plan_host(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_tokens, int32_t num_parts,
+                  int32_t *segments, int32_t *counts, int32_t cap);
+
+/*
+ * Synchronises `stream`, reads the workspace's device error word into *flags
+ * (KVD_DEVERR_* bits) and clears it.  Returns KVD_OK, KVD_ERR_DEVICE when any
+ * flag was set, or KVD_ERR_CUDA.
+ */
+int kvd_read_device_error(void *workspace, kvd_stream_t stream, uint32_t *flags);
+
+/*
+ * Test knobs, process-wide, read at launch time; not for production use.
+ *   KVD_DEBUG_WAIT_LIMIT_NS    limit of one bounded pipeline wait (default 2e9 ns)
+ *   KVD_DEBUG_SKIP_FIRST_LOAD  nonzero: the first tile's copy is never issued, so
+ *                              the consumers' bounded wait runs out and the call
+ *                              reports KVD_DEVERR_TIMEOUT (exercises the timeout
+ *                              path without any fault)
+ */
+enum { KVD_DEBUG_WAIT_LIMIT_NS = 1, KVD_DEBUG_SKIP_FIRST_LOAD = 2 };
+int kvd_debug_set(int knob, long long value);
+
+/*
+ * Measurement hook, process-wide: when both are non-null (cudaEvent_t handles),
+ * every decode call records `before_main` on its stream just before launching
+ * its main decode kernel and `after_main` just after it, so that a benchmark can
+ * time that kernel alone with events.  Pass NULLs to turn it off.
+ */
+int kvd_profile_events(void *before_main, void *after_main);
+
+/* Number of SMs of the current device (the default part count), or a negative code. */
+int kvd_num_sms(void);
+
+/* Static description of a status code. */
+const char *kvd_status_string(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int kvd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVDECODE_H */

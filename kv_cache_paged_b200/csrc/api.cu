@@ -1,0 +1,349 @@
+// C-ABI entry points: validation, workspace sizing, TMA descriptors, launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "kvdecode.h"
+
+using namespace kvd;
+
+namespace {
+
+// Dynamic shared memory the decode kernels may ask for (the SM's 227 KB less
+// the static arrays and the 1 KB alignment slack).
+constexpr size_t SMEM_BUDGET = 220 * 1024;
+
+std::atomic<int> g_debug_flags{0};
+std::atomic<void *> g_ev_before{nullptr}, g_ev_after{nullptr};
+
+void record(std::atomic<void *> &ev, cudaStream_t st) {
+    void *e = ev.load();
+    if (e && g_ev_before.load() && g_ev_after.load()) cudaEventRecord((cudaEvent_t)e, st);
+}
+std::atomic<long long> g_wait_limit_ns{(long long)WAIT_LIMIT_NS};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    });
+    return fn;
+}
+
+bool encode(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
+            const cuuint32_t *box, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms_current() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < 64) cache[dev] = n;
+    return n;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ----------------------------------------------------------------------------- GQA / GTA
+struct GroupPlan {
+    int gpc, n_sub, parts, nt, nstage;
+    uint32_t stage_bytes, stage_bytes_tx;
+    size_t ws_bytes;
+};
+
+// Shared validation and sizing for the GQA/GTA kernel.  tied: GTA.
+int plan_group(bool tied, const void *q, const void *c0, const void *c1, const int32_t *bt, const int32_t *sl,
+               const void *out, const float *lse, int B, int L, int h_q, int h_kv, int d, int d_r, int S, int P,
+               int max_pages, float scale, int num_parts, GroupPlan *gp) {
+    if (B < 0 || L < 1 || h_q < 1 || h_kv < 1 || S < 1 || P < 1 || max_pages < 1 || num_parts < 0)
+        return KVD_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return KVD_ERR_INVALID_ARG;
+    if (h_q % h_kv) return KVD_ERR_INVALID_ARG;
+    if (!q || !c0 || !c1 || !bt || !sl || !out || !lse) return KVD_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(c0, 16) || !aligned(c1, 16) || !aligned(out, 4) || !aligned(lse, 4) ||
+        !aligned(bt, 4) || !aligned(sl, 4))
+        return KVD_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return KVD_ERR_UNSUPPORTED_SHAPE;
+    if (tied) {
+        if ((d_r != 32 && d_r != 64) || d_r > d || (d - d_r) % 16) return KVD_ERR_UNSUPPORTED_SHAPE;
+    }
+    if (S % TILE) return KVD_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)P * S >= (1ll << 31) || (long long)max_pages * S >= (1ll << 31)) return KVD_ERR_UNSUPPORTED_SHAPE;
+    const int R = (h_q / h_kv) * L;
+    int nt = R <= 8 ? 1 : R <= 16 ? 2 : R <= 32 ? 4 : 0;
+    if (!nt) return KVD_ERR_UNSUPPORTED_SHAPE;
+    int gpc = 1;
+    for (int g = 8; g >= 1; --g)
+        if (h_kv % g == 0) {
+            gpc = g;
+            break;
+        }
+    const uint32_t kv_tile = (uint32_t)gpc * d * TILE * 2;
+    const uint32_t tx = tied ? kv_tile + TILE * d_r * 2 : 2 * kv_tile;
+    const uint32_t stage = (uint32_t)round_up(tx, 1024);
+    int nstage = (int)((SMEM_BUDGET - 1024) / stage);
+    if (nstage > MAX_STAGES) nstage = MAX_STAGES;
+    if (nstage < 2) return KVD_ERR_UNSUPPORTED_SHAPE;
+    const int n_sub = h_kv / gpc;
+    int parts = num_parts;
+    if (parts == 0) {
+        const int sms = num_sms_current();
+        if (sms <= 0) return KVD_ERR_CUDA;
+        parts = sms / n_sub > 0 ? sms / n_sub : 1;
+    }
+    const size_t slots = (size_t)B + parts - 1;
+    const size_t rows = (size_t)L * h_q;
+    gp->gpc = gpc;
+    gp->n_sub = n_sub;
+    gp->parts = parts;
+    gp->nt = nt;
+    gp->nstage = nstage;
+    gp->stage_bytes = stage;
+    gp->stage_bytes_tx = tx;
+    gp->ws_bytes = WS_HEADER + round_up(slots * rows * 4, 256) + slots * rows * d * 4;
+    return KVD_OK;
+}
+
+int run_group(bool tied, const void *q, const void *c0, const void *c1, const int32_t *bt, const int32_t *sl,
+              void *out, float *lse, int B, int L, int h_q, int h_kv, int d, int d_r, int S, int P, int max_pages,
+              float scale, int num_parts, void *ws, size_t ws_bytes, cudaStream_t st) {
+    GroupPlan gp;
+    int rc = plan_group(tied, q, c0, c1, bt, sl, out, lse, B, L, h_q, h_kv, d, d_r, S, P, max_pages, scale,
+                        num_parts, &gp);
+    if (rc != KVD_OK) return rc;
+    if (!ws || !aligned(ws, 256)) return KVD_ERR_INVALID_ARG;
+    if (ws_bytes < gp.ws_bytes) return KVD_ERR_WORKSPACE_TOO_SMALL;
+    if (B == 0) return KVD_OK;
+
+    CUtensorMap m0, m1;
+    const cuuint64_t tokens = (cuuint64_t)P * S;
+    {
+        cuuint64_t dims[3] = {64, tokens, (cuuint64_t)h_kv * d / 64};
+        cuuint64_t strides[2] = {(cuuint64_t)h_kv * d * 2, 128};
+        cuuint32_t box[3] = {64, (cuuint32_t)TILE, (cuuint32_t)(gp.gpc * d / 64)};
+        if (!encode(&m0, c0, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+        if (!tied && !encode(&m1, c1, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+    }
+    if (tied) {
+        cuuint64_t dims[2] = {(cuuint64_t)d_r, tokens};
+        cuuint64_t strides[1] = {(cuuint64_t)d_r * 2};
+        cuuint32_t box[2] = {(cuuint32_t)d_r, (cuuint32_t)TILE};
+        if (!encode(&m1, c1, 2, dims, strides, box,
+                    d_r == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+            return KVD_ERR_CUDA;
+    }
+
+    const size_t slots = (size_t)B + gp.parts - 1;
+    const size_t rows = (size_t)L * h_q;
+    uint8_t *w = (uint8_t *)ws;
+    GroupArgs a;
+    a.q = (const __nv_bfloat16 *)q;
+    a.block_table = bt;
+    a.seqlens = sl;
+    a.out = (__nv_bfloat16 *)out;
+    a.lse = lse;
+    a.err = (uint32_t *)w;
+    a.ws_lse = (float *)(w + WS_HEADER);
+    a.ws_o = (float *)(w + WS_HEADER + round_up(slots * rows * 4, 256));
+    a.B = B;
+    a.L = L;
+    a.h_q = h_q;
+    a.h_kv = h_kv;
+    a.page_size = S;
+    a.num_pages = P;
+    a.max_pages = max_pages;
+    a.gpc = gp.gpc;
+    a.n_sub = gp.n_sub;
+    a.parts = gp.parts;
+    a.nstage = gp.nstage;
+    a.stage_bytes = gp.stage_bytes;
+    a.stage_bytes_tx = gp.stage_bytes_tx;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
+    a.debug_flags = g_debug_flags.load();
+    const size_t smem = (size_t)gp.nstage * gp.stage_bytes + 1024;
+    record(g_ev_before, st);
+    cudaError_t e = launch_group_decode(tied, d, tied ? d_r : 0, gp.nt, m0, m1, a, gp.parts * gp.n_sub, smem, st);
+    if (e != cudaSuccess) return KVD_ERR_CUDA;
+    record(g_ev_after, st);
+
+    CombineArgs c;
+    c.seqlens = sl;
+    c.ws_lse = a.ws_lse;
+    c.ws_o = a.ws_o;
+    c.out = (__nv_bfloat16 *)out;
+    c.lse = lse;
+    c.B = B;
+    c.L = L;
+    c.tile = TILE;
+    c.max_tokens = max_pages * S;
+    c.parts = gp.parts;
+    c.rows = (int)rows;
+    c.d_v = d;
+    if (launch_combine(c, st) != cudaSuccess) return KVD_ERR_CUDA;
+    return KVD_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kvd_gqa_workspace_size(const kvd_gqa_params *p) {
+    if (!p) return 0;
+    GroupPlan gp;
+    if (plan_group(false, p->q, p->k_cache, p->v_cache, p->block_table, p->seqlens, p->out, p->lse, p->B, p->L,
+                   p->h_q, p->h_kv, p->d, 0, p->page_size, p->num_pages, p->max_pages, p->scale, p->num_parts,
+                   &gp) != KVD_OK)
+        return 0;
+    return gp.ws_bytes;
+}
+
+size_t kvd_gta_workspace_size(const kvd_gta_params *p) {
+    if (!p) return 0;
+    GroupPlan gp;
+    if (plan_group(true, p->q, p->tied_cache, p->rope_cache, p->block_table, p->seqlens, p->out, p->lse, p->B,
+                   p->L, p->h_q, p->h_kv, p->d_h, p->d_r, p->page_size, p->num_pages, p->max_pages, p->scale,
+                   p->num_parts, &gp) != KVD_OK)
+        return 0;
+    return gp.ws_bytes;
+}
+
+int kvd_gqa_decode(const kvd_gqa_params *p, void *ws, size_t ws_bytes, kvd_stream_t stream) {
+    if (!p) return KVD_ERR_INVALID_ARG;
+    return run_group(false, p->q, p->k_cache, p->v_cache, p->block_table, p->seqlens, p->out, p->lse, p->B, p->L,
+                     p->h_q, p->h_kv, p->d, 0, p->page_size, p->num_pages, p->max_pages, p->scale, p->num_parts, ws,
+                     ws_bytes, (cudaStream_t)stream);
+}
+
+int kvd_gta_decode(const kvd_gta_params *p, void *ws, size_t ws_bytes, kvd_stream_t stream) {
+    if (!p) return KVD_ERR_INVALID_ARG;
+    return run_group(true, p->q, p->tied_cache, p->rope_cache, p->block_table, p->seqlens, p->out, p->lse, p->B,
+                     p->L, p->h_q, p->h_kv, p->d_h, p->d_r, p->page_size, p->num_pages, p->max_pages, p->scale,
+                     p->num_parts, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_tokens, int32_t num_parts,
+             int32_t *segments, int32_t *counts, int32_t cap, kvd_stream_t stream) {
+    if (B < 0 || tile < 1 || max_tokens < 0 || num_parts < 1 || cap < 0) return KVD_ERR_INVALID_ARG;
+    if ((B > 0 && !seqlens) || !counts || (cap > 0 && !segments)) return KVD_ERR_INVALID_ARG;
+    return launch_plan(seqlens, B, tile, max_tokens, 1, num_parts, segments, counts, cap, (cudaStream_t)stream) ==
+                   cudaSuccess
+               ? KVD_OK
+               : KVD_ERR_CUDA;
+}
+
+int kvd_plan_host(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_tokens, int32_t num_parts,
+                  int32_t *segments, int32_t *counts, int32_t cap) {
+    if (B < 0 || tile < 1 || max_tokens < 0 || num_parts < 1 || cap < 0) return KVD_ERR_INVALID_ARG;
+    if ((B > 0 && !seqlens) || !counts || (cap > 0 && !segments)) return KVD_ERR_INVALID_ARG;
+    int64_t N = 0;
+    for (int b = 0; b < B; ++b) N += tiles_of(clamp_len(seqlens[b], max_tokens, 1, nullptr), tile);
+    const int64_t P = N < num_parts ? N : num_parts;
+    for (int c = 0; c < num_parts; ++c) {
+        int cnt = 0;
+        if (N > 0 && c < P) {
+            const int64_t lo = part_begin(c, N, P), hi = part_begin(c + 1, N, P);
+            int64_t cu = 0;
+            for (int b = 0; b < B && cu < hi; ++b) {
+                const int32_t n = tiles_of(clamp_len(seqlens[b], max_tokens, 1, nullptr), tile);
+                if (n > 0 && cu < hi && cu + n > lo) {
+                    if (cnt < cap) {
+                        Seg s = make_seg(b, cu, n, lo, hi, c, N, P);
+                        int32_t *o = segments + ((size_t)c * cap + cnt) * 6;
+                        o[0] = s.b;
+                        o[1] = s.t0;
+                        o[2] = s.t1;
+                        o[3] = s.split;
+                        o[4] = s.nsplit;
+                        o[5] = s.slot;
+                    }
+                    ++cnt;
+                }
+                cu += n;
+            }
+        }
+        counts[c] = cnt;
+    }
+    return KVD_OK;
+}
+
+int kvd_read_device_error(void *ws, kvd_stream_t stream, uint32_t *flags) {
+    if (!ws || !flags) return KVD_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess) return KVD_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof v, st) != cudaSuccess) return KVD_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KVD_ERR_CUDA;
+    *flags = v;
+    return v ? KVD_ERR_DEVICE : KVD_OK;
+}
+
+int kvd_profile_events(void *before_main, void *after_main) {
+    if ((before_main == nullptr) != (after_main == nullptr)) return KVD_ERR_INVALID_ARG;
+    g_ev_before.store(before_main);
+    g_ev_after.store(after_main);
+    return KVD_OK;
+}
+
+int kvd_num_sms(void) {
+    const int n = num_sms_current();
+    return n > 0 ? n : KVD_ERR_CUDA;
+}
+
+int kvd_debug_set(int knob, long long value) {
+    switch (knob) {
+        case KVD_DEBUG_WAIT_LIMIT_NS:
+            if (value <= 0) return KVD_ERR_INVALID_ARG;
+            g_wait_limit_ns.store(value);
+            return KVD_OK;
+        case KVD_DEBUG_SKIP_FIRST_LOAD:
+            if (value)
+                g_debug_flags.fetch_or(DEBUG_SKIP_FIRST_LOAD);
+            else
+                g_debug_flags.fetch_and(~DEBUG_SKIP_FIRST_LOAD);
+            return KVD_OK;
+        default:
+            return KVD_ERR_INVALID_ARG;
+    }
+}
+
+const char *kvd_status_string(int s) {
+    switch (s) {
+        case KVD_OK: return "ok";
+        case KVD_ERR_INVALID_ARG: return "invalid argument";
+        case KVD_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case KVD_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case KVD_ERR_CUDA: return "CUDA error";
+        case KVD_ERR_DEVICE: return "device error flag set";
+        default: return "unknown status";
+    }
+}
+
+int kvd_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,270 @@
+// Shared device helpers for the decode kernels: PTX wrappers (mbarrier, TMA,
+// ldmatrix, mma.sync, movmatrix), bounded waits, error flags and the split plan.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvd {
+
+constexpr uint32_t DEVERR_TIMEOUT = 1u;
+constexpr uint32_t DEVERR_BAD_PAGE = 2u;
+constexpr uint32_t DEVERR_BAD_SEQLEN = 4u;
+
+// Workspace layout: [0, 256) header (error word at 0); then partial lse, then partial O.
+constexpr size_t WS_HEADER = 256;
+
+// Tokens per pipeline tile for the warp-MMA kernels (one m16 row block).
+constexpr int TILE = 16;
+
+// Default limit for one pipeline wait before the kernel gives up (ns).
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
+// ----------------------------------------------------------------------------- split plan
+// The (sequence, tile) stream is the concatenation over b of ceil(T_b / tile)
+// tiles, N in all.  It is cut into P = min(parts, N) parts; part c < P covers
+// tiles [floor(c N / P), floor((c+1) N / P)), so every part is non-empty and
+// the parts holding one sequence's tiles are consecutive.  Parts c >= P are idle.
+struct Seg {
+    int32_t b, t0, t1, split, nsplit, slot;
+};
+
+__host__ __device__ inline int64_t part_begin(int64_t c, int64_t N, int64_t parts) { return (c * N) / parts; }
+
+// The part containing tile x (0 <= x < N): the largest c with part_begin(c) <= x.
+__host__ __device__ inline int64_t part_of(int64_t x, int64_t N, int64_t parts) {
+    return ((x + 1) * parts - 1) / N;
+}
+
+// Clamp a sequence length to [0, max_tokens]; report whether it needed it.
+__host__ __device__ inline int32_t clamp_len(int32_t T, int32_t max_tokens, int32_t L, bool *bad) {
+    bool b = (T < 0) || (T > max_tokens) || (T > 0 && T < L);
+    if (bad) *bad = b;
+    if (T < 0) return 0;
+    if (T > max_tokens) return max_tokens;
+    return T;
+}
+
+__host__ __device__ inline int32_t tiles_of(int32_t T, int32_t tile) { return (T + tile - 1) / tile; }
+
+// Fill `seg` for sequence b whose tiles are [cu, cu + n) intersected with part c's range.
+__host__ __device__ inline Seg make_seg(int32_t b, int64_t cu, int32_t n, int64_t lo, int64_t hi, int64_t c,
+                                        int64_t N, int64_t parts) {
+    Seg s;
+    s.b = b;
+    int64_t a = lo > cu ? lo : cu;
+    int64_t e = hi < cu + n ? hi : cu + n;
+    s.t0 = (int32_t)(a - cu);
+    s.t1 = (int32_t)(e - cu);
+    int64_t first = part_of(cu, N, parts);
+    int64_t last = part_of(cu + n - 1, N, parts);
+    s.split = (int32_t)(c - first);
+    s.nsplit = (int32_t)(last - first + 1);
+    s.slot = (int32_t)(b + c);
+    return s;
+}
+
+#ifdef __CUDACC__
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void set_error(uint32_t *err, uint32_t bits) {
+    if (err) atomicOr(err, bits);
+}
+
+// Warp-cooperative plan walk.  Every lane of the calling warp must call it with
+// the same arguments.  Calls emit(seg) on lane 0 for each segment of part c, in
+// order, up to the end of the part; returns N (total tiles).
+template <typename Emit>
+__device__ __forceinline__ int64_t plan_walk(const int32_t *__restrict__ seqlens, int32_t B, int32_t tile,
+                                             int32_t max_tokens, int32_t L, int64_t c, int64_t parts,
+                                             uint32_t *err, Emit emit) {
+    const int lane = threadIdx.x & 31;
+    int64_t N = 0;
+    for (int32_t base = 0; base < B; base += 32) {
+        int32_t b = base + lane;
+        int32_t n = 0;
+        if (b < B) {
+            bool bad;
+            int32_t T = clamp_len(__ldg(seqlens + b), max_tokens, L, &bad);
+            if (bad && c == 0) set_error(err, DEVERR_BAD_SEQLEN);
+            n = tiles_of(T, tile);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+        N += n;
+    }
+    if (N == 0) return 0;
+    if (parts > N) parts = N;
+    if (c >= parts) return N;
+    const int64_t lo = part_begin(c, N, parts), hi = part_begin(c + 1, N, parts);
+    if (lo >= hi) return N;
+    int64_t run = 0;
+    for (int32_t base = 0; base < B && run < hi; base += 32) {
+        int32_t b = base + lane;
+        int32_t n = 0;
+        if (b < B) n = tiles_of(clamp_len(__ldg(seqlens + b), max_tokens, L, nullptr), tile);
+        int32_t incl = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int64_t cu = run + (incl - n);
+        bool hit = (b < B) && n > 0 && cu < hi && cu + n > lo;
+        uint32_t mask = __ballot_sync(0xffffffffu, hit);
+        while (mask) {
+            int src = __ffs(mask) - 1;
+            mask &= mask - 1;
+            int64_t cu_s = __shfl_sync(0xffffffffu, cu, src);
+            int32_t n_s = __shfl_sync(0xffffffffu, n, src);
+            if (lane == 0) emit(make_seg(base + src, cu_s, n_s, lo, hi, c, N, parts));
+        }
+        run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return N;
+}
+
+// ----------------------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait, by all 32 lanes of a warp together, for phase `parity` of `bar` to
+// complete.  Every lane gets the same answer.  Gives up (returns false) when
+// *abort becomes nonzero or after limit_ns; on running out it records
+// DEVERR_TIMEOUT in *err (when err is not null) and raises *abort so that the
+// other warps stop too.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *err,
+                                               uint64_t limit_ns) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+        int stop = 0;
+        if ((threadIdx.x & 31) == 0) {
+            if (*abort) {
+                stop = 1;
+            } else if (globaltimer() - t0 > limit_ns) {
+                set_error(err, DEVERR_TIMEOUT);
+                *abort = 1;
+                stop = 1;
+            }
+        }
+        if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+    }
+}
+
+// ----------------------------------------------------------------------------- TMA
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *m, uint64_t *bar, int x, int y,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(m), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uint64_t *bar, int x, int y, int z,
+                                            uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_u32(dst)),
+        "l"(m), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
+        : "memory");
+}
+// L2 policy for data read exactly once (the KV stream).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// ----------------------------------------------------------------------------- warp MMA
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+// D = A(16x16, row) * B(16x8, col) + D, bf16 in, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Transpose an 8x8 b16 matrix held one bf16x2 per lane in fragment order.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+// Pack two fp32 into bf16x2 (round to nearest even): lo -> bits [0,16), hi -> [16,32).
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 128-byte-swizzled tile of 128-byte rows (TMA SWIZZLE_128B): byte offset of
+// 16-byte chunk k of row r.  The tile base must be 1024-byte aligned.
+__device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t k) { return r * 128u + ((k ^ (r & 7u)) << 4); }
+// 64-byte rows, TMA SWIZZLE_64B (address bits [4,6) ^= bits [7,9)).
+__device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t k) {
+    uint32_t off = r * 64u + k * 16u;
+    return off ^ (((off >> 7) & 3u) << 4);
+}
+
+// Programmatic dependent launch.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+#endif  // __CUDACC__
+
+}  // namespace kvd

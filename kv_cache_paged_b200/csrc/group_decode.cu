@@ -1,0 +1,390 @@
+// GQA and GTA decode over a paged KV cache: warp-level tensor-core kernel.
+//
+// "Hardware-Efficient Attention for Fast Decoding", section 3: with g_q query
+// heads per KV head the decode step does about 2 g_q / m_kv FLOPs per loaded
+// byte (about 4 for GQA and 7.5 for GTA at h_q = 32, h_kv = 8), far below the
+// B200 ridge, so this kernel is built to stream the cache at HBM speed; the
+// math uses mma.sync because g_q * q_len (4 rows per group) is far too small
+// for a 128-row tcgen05 tile.
+//
+// One CTA owns one contiguous part of the (sequence, 16-token tile) stream and
+// `gpc` KV groups.  Warp `gpc` is the producer: it resolves block-table entries
+// for a whole warp's worth of pages at once and issues one TMA per operand per
+// tile (128-byte swizzle) into an n-stage mbarrier ring.  Warps 0..gpc-1 each
+// own one KV group; per tile they compute S^T = K q^T with tokens as the MMA's
+// M dimension (so the 4 query rows only pad N = 8, not M = 16), run the online
+// softmax in fp32 (base 2, scale folded in), transpose P with movmatrix into
+// the B operand and accumulate O^T += V^T P^T (V^T via ldmatrix.trans).  GTA
+// reads the tied tile twice from shared memory: its first d_h - d_r dims as the
+// key and all d_h dims as the value; the shared rope tile supplies the rest of
+// the key.  Sequences cut into several parts write fp32 partials that the
+// combine kernel merges.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvd {
+
+namespace {
+
+constexpr int MAXSEG = 128;
+
+template <bool TIED, int D, int DR, int NT>
+__global__ void __launch_bounds__(9 * 32, 1)
+    group_decode_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
+                        const GroupArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
+    __shared__ Seg segs[MAXSEG];
+    __shared__ int nseg_sh, more_sh;
+    __shared__ volatile int abort_sh;
+
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gpc = a.gpc;
+    const int part = blockIdx.x / a.n_sub, sub = blockIdx.x % a.n_sub;
+    const int nstage = a.nstage;
+    const int g_q = a.h_q / a.h_kv;
+    const int R = g_q * a.L;
+    const int max_tokens = a.max_pages * a.page_size;
+    const uint32_t kv_tile = (uint32_t)(gpc * D * TILE * 2);  // bytes of one K / V / tied tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nstage; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], gpc);
+        }
+        abort_sh = 0;
+        fence_mbar_init();
+    }
+    if (warp == gpc && lane == 0) {
+        tma_prefetch_desc(&map0);
+        tma_prefetch_desc(&map1);
+    }
+    pdl_launch_dependents();
+    __syncthreads();
+
+    uint32_t it = 0;  // tile counter, identical in every warp
+    for (int skip = 0;; skip += MAXSEG) {
+        if (warp == gpc) {
+            int cnt = 0;
+            plan_walk(a.seqlens, a.B, TILE, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
+                if (cnt >= skip && cnt < skip + MAXSEG) segs[cnt - skip] = s;
+                ++cnt;
+            });
+            if (lane == 0) {
+                nseg_sh = cnt - skip < MAXSEG ? (cnt - skip > 0 ? cnt - skip : 0) : MAXSEG;
+                more_sh = cnt > skip + MAXSEG;
+            }
+        }
+        __syncthreads();
+        const int nseg = nseg_sh;
+
+        if (warp == gpc) {
+            // ------------------------------------------------------------ producer
+            const uint64_t pol = policy_evict_first();
+            const int z0 = sub * gpc * (D / 64);  // first 64-wide chunk of this CTA's groups
+            uint32_t issued = it;
+            bool stop = false;
+            for (int si = 0; si < nseg && !stop; ++si) {
+                const Seg sg = segs[si];
+                const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
+                const int tiles_per_page = a.page_size / TILE;
+                const int p_first = sg.t0 / tiles_per_page;
+                const int p_last = (sg.t1 - 1) / tiles_per_page;
+                for (int pb = p_first; pb <= p_last && !stop; pb += 32) {
+                    // distributed offset calculation: one block-table entry per lane
+                    int page = 0;
+                    if (pb + lane <= p_last) {
+                        page = __ldg(bt + pb + lane);
+                        if (page < 0 || page >= a.num_pages) {
+                            set_error(a.err, DEVERR_BAD_PAGE);
+                            page = 0;
+                        }
+                    }
+                    const int t_lo = max(sg.t0, pb * tiles_per_page);
+                    const int t_hi = min(sg.t1, (pb + 32) * tiles_per_page);
+                    for (int t = t_lo; t < t_hi; ++t) {
+                        const int pg = __shfl_sync(0xffffffffu, page, t / tiles_per_page - pb);
+                        const uint32_t stage = issued % nstage;
+                        if (!mbar_wait_warp(&empty_bar[stage], ((issued / nstage) & 1) ^ 1, &abort_sh, a.err,
+                                            a.wait_limit_ns)) {
+                            stop = true;
+                            break;
+                        }
+                        if (lane == 0) {
+                            uint8_t *st = smem + (size_t)stage * a.stage_bytes;
+                            const int row = pg * a.page_size + (t % tiles_per_page) * TILE;
+                            mbar_arrive_expect_tx(&full_bar[stage], a.stage_bytes_tx);
+                            if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || issued != 0) {
+                                tma_load_3d(st, &map0, &full_bar[stage], 0, row, z0, pol);
+                                if (TIED)
+                                    tma_load_2d(st + kv_tile, &map1, &full_bar[stage], 0, row, pol);
+                                else
+                                    tma_load_3d(st + kv_tile, &map1, &full_bar[stage], 0, row, z0, pol);
+                            }
+                        }
+                        ++issued;
+                    }
+                }
+            }
+            if (stop) {
+                // Let every copy already issued land before the CTA can exit.
+                const uint32_t lo = issued > (uint32_t)nstage ? issued - nstage : 0;
+                for (uint32_t k = lo; k < issued; ++k) {
+                    volatile int never = 0;
+                    mbar_wait_warp(&full_bar[k % nstage], (k / nstage) & 1, &never, nullptr, a.wait_limit_ns);
+                }
+            }
+            it = issued;
+        } else {
+            // ------------------------------------------------------------ consumers
+            const int gl = warp;                      // local group
+            const int g = sub * gpc + gl;             // KV group
+            const int lr = lane >> 2, lc = lane & 3;  // fragment row / column-pair
+            for (int si = 0; si < nseg; ++si) {
+                const Seg sg = segs[si];
+                const int b = sg.b;
+                const int T = clamp_len(__ldg(a.seqlens + b), max_tokens, a.L, nullptr);
+
+                // q^T as B fragments: rows n = 8 nt + lr, dims kk*16 + 2 lc (+8)
+                uint32_t qf[NT][D / 16][2];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int n = 8 * nt + lr;
+                    if (n < R) {
+                        const int i = n / g_q, head = g * g_q + n % g_q;
+                        const uint32_t *qp =
+                            (const uint32_t *)(a.q + (((size_t)b * a.L + i) * a.h_q + head) * D);
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            qf[nt][kk][0] = __ldg(qp + kk * 8 + lc);
+                            qf[nt][kk][1] = __ldg(qp + kk * 8 + 4 + lc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) qf[nt][kk][0] = qf[nt][kk][1] = 0u;
+                    }
+                }
+                // causal limit of the two rows this lane's accumulators hold
+                int lim[NT][2];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int n = 8 * nt + 2 * lc + j;
+                        lim[nt][j] = n < R ? T - a.L + n / g_q : -1;
+                    }
+
+                float m[NT][2], l[NT][2], o[NT][D / 16][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    m[nt][0] = m[nt][1] = -INFINITY;
+                    l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+                    for (int mt = 0; mt < D / 16; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
+                }
+
+                bool ok = true;
+                for (int tile = sg.t0; tile < sg.t1; ++tile, ++it) {
+                    const uint32_t stage = it % nstage;
+                    if (!mbar_wait_warp(&full_bar[stage], (it / nstage) & 1, &abort_sh, a.err, a.wait_limit_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t base = smem_u32(smem + (size_t)stage * a.stage_bytes);
+                    const int tok0 = tile * TILE;
+
+                    // ---- S^T = K q^T (tokens x rows)
+                    float s[NT][4];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+                    {
+                        const int mi = lane >> 3;
+                        const int tk = (lane & 7) + 8 * (mi & 1);
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int dim = kk * 16 + 8 * (mi >> 1);
+                            uint32_t addr;
+                            if (!TIED || kk * 16 < D - DR) {
+                                const int row = (gl * (D / 64) + dim / 64) * TILE + tk;
+                                addr = base + sw128(row, (dim & 63) >> 3);
+                            } else {
+                                const int rd = dim - (D - DR);
+                                addr = base + kv_tile + (DR == 64 ? sw128(tk, rd >> 3) : sw64(tk, rd >> 3));
+                            }
+                            uint32_t A[4];
+                            ldsm_x4(addr, A);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) mma_bf16(s[nt], A, qf[nt][kk][0], qf[nt][kk][1]);
+                        }
+                    }
+
+                    // ---- mask, online softmax (base 2)
+                    const int ta = tok0 + lr, tb = ta + 8;
+                    float alpha[NT][2];
+                    bool rescale = false;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            float v0 = ta <= lim[nt][j] ? s[nt][j] * a.scale_log2 : -INFINITY;
+                            float v1 = tb <= lim[nt][j] ? s[nt][2 + j] * a.scale_log2 : -INFINITY;
+                            float mx = fmaxf(v0, v1);
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                            const float m_new = fmaxf(m[nt][j], mx);
+                            // nothing visible yet: O and l are still 0, leave them alone
+                            float al = 1.f, p0 = 0.f, p1 = 0.f;
+                            if (m_new != -INFINITY) {
+                                al = ex2(m[nt][j] - m_new);
+                                p0 = ex2(v0 - m_new);
+                                p1 = ex2(v1 - m_new);
+                            }
+                            m[nt][j] = m_new;
+                            l[nt][j] = l[nt][j] * al + p0 + p1;
+                            s[nt][j] = p0;
+                            s[nt][2 + j] = p1;
+                            alpha[nt][j] = al;
+                            rescale |= (al != 1.f);
+                        }
+                    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int mt = 0; mt < D / 16; ++mt) {
+                                o[nt][mt][0] *= alpha[nt][0];
+                                o[nt][mt][1] *= alpha[nt][1];
+                                o[nt][mt][2] *= alpha[nt][0];
+                                o[nt][mt][3] *= alpha[nt][1];
+                            }
+                    }
+
+                    // ---- P^T as B fragments (tokens x rows), via an 8x8 transpose per half
+                    uint32_t pb[NT][2];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        pb[nt][0] = movmatrix_t(pack_bf16(s[nt][0], s[nt][1]));
+                        pb[nt][1] = movmatrix_t(pack_bf16(s[nt][2], s[nt][3]));
+                    }
+
+                    // ---- O^T += V^T P^T; tokens past T_b hold garbage (NaN poison): zero them
+                    const bool tail = tok0 + TILE > T;
+                    uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
+                    if (tail) {
+                        const int t0 = tok0 + 2 * lc;
+                        mlo = (t0 < T ? 0x0000ffffu : 0u) | (t0 + 1 < T ? 0xffff0000u : 0u);
+                        mhi = (t0 + 8 < T ? 0x0000ffffu : 0u) | (t0 + 9 < T ? 0xffff0000u : 0u);
+                    }
+                    {
+                        const int mi = lane >> 3;
+                        const int tk = (lane & 7) + 8 * (mi >> 1);
+                        const uint32_t vbase = TIED ? base : base + kv_tile;
+#pragma unroll
+                        for (int mt = 0; mt < D / 16; ++mt) {
+                            const int dim = mt * 16 + 8 * (mi & 1);
+                            const int row = (gl * (D / 64) + dim / 64) * TILE + tk;
+                            uint32_t A[4];
+                            ldsm_x4_t(vbase + sw128(row, (dim & 63) >> 3), A);
+                            A[0] &= mlo;
+                            A[1] &= mlo;
+                            A[2] &= mhi;
+                            A[3] &= mhi;
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) mma_bf16(o[nt][mt], A, pb[nt][0], pb[nt][1]);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty_bar[stage]);
+                }
+                if (!ok) {
+                    // skip the rest; keep the tile counter in step with the producer
+                    break;
+                }
+
+                // ---- epilogue
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        float v = l[nt][j];
+                        v += __shfl_xor_sync(0xffffffffu, v, 4);
+                        v += __shfl_xor_sync(0xffffffffu, v, 8);
+                        v += __shfl_xor_sync(0xffffffffu, v, 16);
+                        l[nt][j] = v;
+                    }
+                const int rows_b = a.L * a.h_q;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int n = 8 * nt + 2 * lc + j;
+                        if (n >= R) continue;
+                        const int i = n / g_q, head = g * g_q + n % g_q;
+                        const float lv = l[nt][j];
+                        const float inv = lv > 0.f ? 1.f / lv : 0.f;
+                        const float lse_v = lv > 0.f ? (m[nt][j] + lg2(lv)) * 0.69314718055994530942f : -INFINITY;
+                        const int r = i * a.h_q + head;
+                        if (sg.nsplit == 1) {
+                            __nv_bfloat16 *op = a.out + ((size_t)b * rows_b + r) * D;
+#pragma unroll
+                            for (int mt = 0; mt < D / 16; ++mt) {
+                                op[mt * 16 + lr] = __float2bfloat16_rn(o[nt][mt][j] * inv);
+                                op[mt * 16 + 8 + lr] = __float2bfloat16_rn(o[nt][mt][2 + j] * inv);
+                            }
+                            if (lr == 0) a.lse[(size_t)b * rows_b + r] = lse_v;
+                        } else {
+                            float *op = a.ws_o + ((size_t)sg.slot * rows_b + r) * D;
+#pragma unroll
+                            for (int mt = 0; mt < D / 16; ++mt) {
+                                op[mt * 16 + lr] = o[nt][mt][j] * inv;
+                                op[mt * 16 + 8 + lr] = o[nt][mt][2 + j] * inv;
+                            }
+                            if (lr == 0) a.ws_lse[(size_t)sg.slot * rows_b + r] = lse_v;
+                        }
+                    }
+            }
+        }
+        __syncthreads();
+        if (!more_sh || abort_sh) break;
+        __syncthreads();
+    }
+}
+
+template <bool TIED, int D, int DR, int NT>
+cudaError_t launch_t(const CUtensorMap &m0, const CUtensorMap &m1, const GroupArgs &a, int grid, size_t smem,
+                     cudaStream_t st) {
+    auto k = group_decode_kernel<TIED, D, DR, NT>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, (a.gpc + 1) * 32, smem, st>>>(m0, m1, a);
+    return cudaGetLastError();
+}
+
+template <bool TIED, int D, int DR>
+cudaError_t launch_nt(int nt, const CUtensorMap &m0, const CUtensorMap &m1, const GroupArgs &a, int grid,
+                      size_t smem, cudaStream_t st) {
+    switch (nt) {
+        case 1: return launch_t<TIED, D, DR, 1>(m0, m1, a, grid, smem, st);
+        case 2: return launch_t<TIED, D, DR, 2>(m0, m1, a, grid, smem, st);
+        case 4: return launch_t<TIED, D, DR, 4>(m0, m1, a, grid, smem, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_group_decode(bool tied, int d, int d_r, int nt, const CUtensorMap &m0, const CUtensorMap &m1,
+                                const GroupArgs &a, int grid, size_t smem, cudaStream_t st) {
+    if (!tied && d == 128) return launch_nt<false, 128, 0>(nt, m0, m1, a, grid, smem, st);
+    if (!tied && d == 64) return launch_nt<false, 64, 0>(nt, m0, m1, a, grid, smem, st);
+    if (tied && d == 128 && d_r == 64) return launch_nt<true, 128, 64>(nt, m0, m1, a, grid, smem, st);
+    if (tied && d == 64 && d_r == 32) return launch_nt<true, 64, 32>(nt, m0, m1, a, grid, smem, st);
+    if (tied && d == 128 && d_r == 32) return launch_nt<true, 128, 32>(nt, m0, m1, a, grid, smem, st);
+    if (tied && d == 64 && d_r == 64) return launch_nt<true, 64, 64>(nt, m0, m1, a, grid, smem, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kvd

@@ -1,0 +1,59 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvd {
+
+constexpr int MAX_STAGES = 8;
+
+// Test knobs (kvd_debug_set): make the first tile's copy never start so that the
+// bounded waits run out, exercising the timeout path without a GPU fault.
+constexpr int DEBUG_SKIP_FIRST_LOAD = 1;
+
+struct GroupArgs {
+    const __nv_bfloat16 *q;
+    const int32_t *block_table;
+    const int32_t *seqlens;
+    __nv_bfloat16 *out;
+    float *lse;
+    float *ws_lse;  // [slots][L * h_q]
+    float *ws_o;    // [slots][L * h_q][d]
+    uint32_t *err;
+    int B, L, h_q, h_kv, page_size, num_pages, max_pages;
+    int gpc;    // KV groups per CTA (consumer warps)
+    int n_sub;  // CTAs per part = h_kv / gpc
+    int parts;
+    int nstage;
+    uint32_t stage_bytes;     // smem bytes per stage (multiple of 1024)
+    uint32_t stage_bytes_tx;  // bytes the TMA copies deliver per stage
+    float scale_log2;         // softmax scale * log2(e)
+    uint64_t wait_limit_ns;
+    int debug_flags;
+};
+
+cudaError_t launch_group_decode(bool tied, int d, int d_r, int nt, const CUtensorMap &m0, const CUtensorMap &m1,
+                                const GroupArgs &a, int grid, size_t smem, cudaStream_t st);
+
+struct CombineArgs {
+    const int32_t *seqlens;
+    const float *ws_lse;
+    const float *ws_o;
+    __nv_bfloat16 *out;
+    float *lse;
+    int B, L, tile, max_tokens, parts;
+    int rows;  // L * h_q
+    int d_v;
+};
+
+// Merges split partials (launched as a programmatic dependent of the decode kernel).
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
+
+// Writes the plan of every part (see kvd_plan).
+cudaError_t launch_plan(const int32_t *seqlens, int B, int tile, int max_tokens, int L, int parts, int32_t *segs,
+                        int32_t *counts, int cap, cudaStream_t st);
+
+}  // namespace kvd

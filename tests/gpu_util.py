@@ -1,0 +1,55 @@
+"""Helpers shared by the GPU tests: move generated inputs to the device, call the
+library through the binding, and compare against the fp64 oracle."""
+import numpy as np
+
+TOL_MAX_ABS = 1e-2    # max |out - oracle| (bf16 inputs, fp32 accumulation)
+TOL_MEAN_ABS = 1e-3   # mean |out - oracle|
+TOL_LSE = 1e-3        # max |lse - oracle|
+
+
+def to_dev(inp, device="cuda"):
+    import torch
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+    d = {"q": bf(inp.q), "block_table": torch.from_numpy(inp.block_table).to(device),
+         "seqlens": torch.from_numpy(inp.seqlens).to(device)}
+    for k, v in inp.caches.items():
+        d[k] = bf(v)
+    return d
+
+
+def run_gpu(inp, dev=None, num_parts=0, workspace=None):
+    from kv_cache_paged_b200 import binding
+    dev = dev if dev is not None else to_dev(inp)
+    if inp.variant == "gqa":
+        out, lse = binding.gqa_decode(dev["q"], dev["k_cache"], dev["v_cache"], dev["block_table"], dev["seqlens"],
+                                      inp.scale, num_parts=num_parts, workspace=workspace)
+    elif inp.variant == "gta":
+        out, lse = binding.gta_decode(dev["q"], dev["tied_cache"], dev["rope_cache"], dev["block_table"],
+                                      dev["seqlens"], inp.scale, num_parts=num_parts, workspace=workspace)
+    else:
+        out, lse = binding.gla_decode(dev["q"], dev["latent_cache"], dev["rope_cache"], dev["block_table"],
+                                      dev["seqlens"], inp.scale, num_parts=num_parts, workspace=workspace)
+    return out, lse
+
+
+def to_np(out, lse):
+    import torch
+    return out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def assert_close(out, lse, ref_out, ref_lse, what=""):
+    """The benchmark spec tolerance: max abs <= 1e-2, mean abs <= 1e-3 on out; |lse| <= 1e-3."""
+    assert out.shape == ref_out.shape, (out.shape, ref_out.shape)
+    assert np.isfinite(out).all(), f"{what}: non-finite output"
+    err = np.abs(out - ref_out)
+    assert err.max() <= TOL_MAX_ABS, f"{what}: max abs err {err.max():.3e}"
+    assert err.mean() <= TOL_MEAN_ABS, f"{what}: mean abs err {err.mean():.3e}"
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(np.isfinite(lse), fin), f"{what}: lse -inf pattern differs"
+    if fin.any():
+        le = np.abs(lse[fin] - ref_lse[fin]).max()
+        assert le <= TOL_LSE, f"{what}: lse err {le:.3e}"
+    return float(err.max()), float(err.mean())

@@ -5,7 +5,7 @@ holds 1.0 in a dimension reserved for h and every other key entry in that
 dimension is 0, while q holds 2^9 there (scale 1/8, so the target scores 64 and
 every other token 0).  The softmax weight of a non-target is e^-64 / (1 + ...)
 < 2e-28, far below bf16 resolution, so out = v_{t*} after rounding.  Values hold
-the target's logical position in base-256 digits, which bf16 represents exactly,
+the target's logical position in base-256 digits (plus one), which bf16 represents exactly,
 so any page or slot addressing error shows up as a wrong integer.
 Slots past T_b and the unreferenced page keep their NaN poison.
 """
@@ -18,7 +18,10 @@ QVAL = wl.f32_to_bf16_bits(np.array([512.0], np.float32))[0]
 
 
 def _digits(t, b):
-    return [t % 256, (t // 256) % 256, b % 256]
+    # digits shifted to 1..256: exact in bf16, and never 0, so the e^-64-weighted
+    # contributions of the other tokens (representable next to 0 in bf16, but not
+    # next to 1 in fp32) cannot show
+    return [t % 256 + 1, (t // 256) % 256 + 1, b % 256 + 1]
 
 
 def make_delta_problem(variant, seed, *, B=3, L=1, h_q=8, h_kv=2, d=32, d_r=16, S=16,

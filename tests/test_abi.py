@@ -1,0 +1,143 @@
+"""The C-ABI library: loads, exports every declared symbol, validates arguments and
+plans splits (host logic only; no GPU needed)."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from kv_cache_paged_b200 import binding
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return binding.lib()
+
+
+def test_every_declared_function_is_exported(lib):
+    names = binding.header_functions()
+    assert len(names) >= 12
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_version(lib):
+    for code, text in binding.STATUS.items():
+        assert lib.kvd_status_string(code).decode() == text
+    assert lib.kvd_version() >= 100
+
+
+def _gta_params(**kw):
+    base = dict(q=16, tied_cache=16, rope_cache=16, block_table=16, seqlens=16, out=16, lse=16,
+                B=2, L=1, h_q=8, h_kv=2, d_h=64, d_r=32, page_size=16, num_pages=10, max_pages=8,
+                scale=0.125, num_parts=4)
+    base.update(kw)
+    return binding.GTAParams(**base)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), -1),                 # null pointer
+    (dict(q=18), -1),                   # misaligned for TMA
+    (dict(h_q=7), -1),                  # h_q % h_kv != 0
+    (dict(L=0), -1),
+    (dict(d_h=96), -2),                 # head dim outside the compiled set
+    (dict(d_r=48), -2),
+    (dict(page_size=24), -2),           # not a multiple of the 16-token tile
+    (dict(h_q=128, h_kv=2, L=1), -2),   # 64 rows per group: beyond the warp-MMA kernel
+    (dict(scale=float("nan")), -1),
+])
+def test_gta_validation_errors(lib, kw, expect):
+    p = _gta_params(**kw)
+    assert lib.kvd_gta_workspace_size(ctypes.byref(p)) == 0
+    assert lib.kvd_gta_decode(ctypes.byref(p), ctypes.c_void_p(256), 1 << 30, None) == expect
+
+
+def test_workspace_size_and_too_small(lib):
+    p = _gta_params()
+    n = lib.kvd_gta_workspace_size(ctypes.byref(p))
+    slots, rows = 2 + 4 - 1, 1 * 8
+    assert n == 256 + ((slots * rows * 4 + 255) // 256) * 256 + slots * rows * 64 * 4
+    assert lib.kvd_gta_decode(ctypes.byref(p), ctypes.c_void_p(256), n - 1, None) == -3
+    assert lib.kvd_gta_decode(ctypes.byref(p), ctypes.c_void_p(8), n, None) == -1   # workspace misaligned
+
+
+def test_gqa_validation(lib):
+    p = binding.GQAParams(q=16, k_cache=16, v_cache=16, block_table=16, seqlens=16, out=16, lse=16,
+                          B=1, L=1, h_q=32, h_kv=8, d=80, page_size=64, num_pages=4, max_pages=4,
+                          scale=0.1, num_parts=2)
+    assert lib.kvd_gqa_decode(ctypes.byref(p), ctypes.c_void_p(256), 1 << 20, None) == -2
+
+
+def test_debug_knobs_validate(lib):
+    assert lib.kvd_debug_set(99, 1) == -1
+    assert lib.kvd_debug_set(binding.DEBUG_WAIT_LIMIT_NS, 0) == -1
+    assert lib.kvd_debug_set(binding.DEBUG_WAIT_LIMIT_NS, 2_000_000_000) == 0
+
+
+# ----------------------------------------------------------------------------- split plan (host copy)
+def _check_plan(seqlens, tile, parts, max_tokens=1 << 30):
+    segs, counts = binding.plan_host(seqlens, tile, max_tokens, parts, cap=max(64, len(seqlens) + 2))
+    tiles = [(-(-int(t) // tile)) for t in seqlens]
+    N = sum(tiles)
+    covered = {b: [] for b in range(len(seqlens))}
+    slots = set()
+    first_part = {}
+    per_part = []
+    for c in range(parts):
+        n = int(counts[c])
+        assert n <= segs.shape[1]
+        ntile = 0
+        prev_b = -1
+        for k in range(n):
+            b, t0, t1, split, nsplit, slot = (int(x) for x in segs[c, k])
+            assert b > prev_b, "segments of a part are in sequence order"
+            prev_b = b
+            assert 0 <= t0 < t1 <= tiles[b]
+            covered[b].append((t0, t1, split, nsplit))
+            assert slot == b + c and slot not in slots
+            assert split == c - first_part.setdefault(b, c)
+            slots.add(slot)
+            ntile += t1 - t0
+        per_part.append(ntile)
+    for b, segs_b in covered.items():
+        segs_b.sort()
+        if tiles[b] == 0:
+            assert segs_b == []
+            continue
+        # contiguous, exact cover of [0, tiles_b), split indices 0..n-1, consistent nsplit
+        assert segs_b[0][0] == 0 and segs_b[-1][1] == tiles[b]
+        for (a0, a1, s0, n0), (b0, b1, s1, n1) in zip(segs_b, segs_b[1:]):
+            assert a1 == b0
+        assert [s[2] for s in segs_b] == list(range(len(segs_b)))
+        assert all(s[3] == len(segs_b) for s in segs_b)
+    if N:
+        busy = per_part[:min(parts, N)]
+        assert min(busy) >= 1, "the first min(parts, N) parts are all non-empty"
+        assert all(x == 0 for x in per_part[min(parts, N):])
+        assert max(busy) - min(busy) <= 1, "parts differ by at most one tile"
+    return per_part
+
+
+@pytest.mark.parametrize("parts", [1, 2, 7, 148, 1000])
+def test_plan_covers_every_tile_once_balanced(parts):
+    rng = np.random.default_rng(parts)
+    sl = rng.integers(1024, 8193, size=32).astype(np.int32)
+    per = _check_plan(sl, 16, parts)
+    assert sum(per) == sum(-(-int(t) // 16) for t in sl)
+
+
+def test_plan_with_empty_and_tiny_sequences():
+    sl = np.array([0, 1, 15, 16, 17, 0, 0, 1000, 0], dtype=np.int32)
+    for parts in (1, 3, 5, 64):
+        _check_plan(sl, 16, parts)
+
+
+def test_plan_all_empty():
+    segs, counts = binding.plan_host(np.zeros(5, np.int32), 16, 1 << 20, 4)
+    assert counts.sum() == 0
+
+
+def test_plan_clamps_oversized_lengths():
+    # lengths above max_tokens are clamped (the decode kernel flags them)
+    segs, counts = binding.plan_host(np.array([100, 5000], np.int32), 16, 256, 2)
+    tiles = sum(int(segs[c, k, 2] - segs[c, k, 1]) for c in range(2) for k in range(counts[c]))
+    assert tiles == 7 + 16
