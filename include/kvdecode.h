@@ -148,6 +148,29 @@ int kvd_gta_decode(const kvd_gta_params *p, void *workspace, size_t workspace_by
 int kvd_gla_decode(const kvd_gla_params *p, void *workspace, size_t workspace_bytes, kvd_stream_t stream);
 
 /*
+ * Allocation-free GTA decode (no counterpart in the paper: an interface for
+ * callers that cannot provide a workspace).  Serving engines that have already
+ * split all of HBM between KV pages and their own arenas cannot allocate more
+ * device memory per call, and code that calls this while a stream is captured
+ * in global mode may not call cudaMalloc at all.  This entry computes exactly
+ * what kvd_gta_decode() computes, with the workspace in a fixed 8 MiB device
+ * array inside the library (held by every GPU that loads the library until the
+ * process exits).  It allocates and frees nothing.
+ *   - The first call on each device looks up that array's device address with
+ *     that device current (and clears its error word); make that first call
+ *     before any stream capture.
+ *   - Calls whose split partials need more than 8 MiB (see
+ *     kvd_gta_workspace_size) are rejected with KVD_ERR_WORKSPACE_TOO_SMALL and
+ *     launch nothing.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; nothing in it needs to start at zero, but calls that overlap on
+ *     the GPU (different streams, no ordering between them) race on it.
+ *   - Device error flags land in the shared array and cannot be read back; use
+ *     kvd_gta_decode() with a workspace to inspect them.
+ */
+int kvd_gta_decode_noalloc(const kvd_gta_params *p, kvd_stream_t stream);
+
+/*
  * Split plan for inspection and tests.  Cuts the (sequence, tile) stream of
  * seqlens[B] (device pointer) with `tile` tokens per tile into num_parts parts
  * exactly as the decode kernels do and writes, for part c, up to `cap` records

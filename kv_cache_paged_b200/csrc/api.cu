@@ -347,3 +347,65 @@ const char *kvd_status_string(int s) {
 int kvd_version(void) { return 100; }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------- allocation-free GTA entry
+// Some callers cannot hand us a workspace: a serving engine that has already
+// carved all of HBM into KV pages and its own arenas (so any further device
+// allocation can fail, or fragment memory it manages), or code that issues
+// this call while a stream is being captured in global mode, where
+// cudaMalloc is not a legal call.  For them kvd_gta_decode_noalloc() runs the
+// same kernels as kvd_gta_decode() with the workspace placed in this fixed
+// device array, which every GPU that loads the library holds until the
+// process exits.
+namespace {
+
+constexpr size_t NOALLOC_WS_BYTES = 8u << 20;  // 8 MiB
+static __device__ __align__(256) uint8_t g_noalloc_ws[NOALLOC_WS_BYTES];
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {nullptr};
+
+// Device address of g_noalloc_ws on the current device.  Host code must not use
+// the symbol itself as a pointer: on the host it names a stand-in, not device
+// memory.  Done once per device, with that device current.
+void *noalloc_workspace(int *status) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) {
+        *status = KVD_ERR_CUDA;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || !p) {
+            *status = KVD_ERR_CUDA;
+            return nullptr;
+        }
+        // The error word at the head of the workspace only collects flags; start it at zero.
+        if (cudaMemset(p, 0, WS_HEADER) != cudaSuccess) {
+            *status = KVD_ERR_CUDA;
+            return nullptr;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *status = KVD_OK;
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int kvd_gta_decode_noalloc(const kvd_gta_params *p, kvd_stream_t stream) {
+    if (!p) return KVD_ERR_INVALID_ARG;
+    GroupPlan gp;
+    int rc = plan_group(true, p->q, p->tied_cache, p->rope_cache, p->block_table, p->seqlens, p->out, p->lse, p->B,
+                        p->L, p->h_q, p->h_kv, p->d_h, p->d_r, p->page_size, p->num_pages, p->max_pages, p->scale,
+                        p->num_parts, &gp);
+    if (rc != KVD_OK) return rc;
+    if (gp.ws_bytes > NOALLOC_WS_BYTES) return KVD_ERR_WORKSPACE_TOO_SMALL;
+    void *ws = noalloc_workspace(&rc);
+    if (rc != KVD_OK) return rc;
+    return run_group(true, p->q, p->tied_cache, p->rope_cache, p->block_table, p->seqlens, p->out, p->lse, p->B,
+                     p->L, p->h_q, p->h_kv, p->d_h, p->d_r, p->page_size, p->num_pages, p->max_pages, p->scale,
+                     p->num_parts, ws, NOALLOC_WS_BYTES, (cudaStream_t)stream);
+}
