@@ -42,7 +42,8 @@
  *                aligned, ZEROED ONCE before its first use (cudaMemset).  It holds
  *                the split-KV partials and a sticky device error word; calls
  *                that overlap on the GPU must not share one workspace.
- * All base pointers must be 16-byte aligned (TMA).
+ * q, caches and (for GLA) out must be 16-byte aligned (TMA, vector stores); out
+ * 8-byte aligned for GQA/GTA; the int32 and fp32 arrays 4-byte aligned.
  *
  * Execution: every entry point is asynchronous on `stream`; there is no host
  * synchronisation and no allocation, so a call can be captured in a CUDA graph.

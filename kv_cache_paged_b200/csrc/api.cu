@@ -71,7 +71,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // ----------------------------------------------------------------------------- GQA / GTA
 struct GroupPlan {
-    int gpc, n_sub, parts, nt, nstage;
+    int gpc, n_sub, parts, nt, nstage, tile;
     uint32_t stage_bytes, stage_bytes_tx;
     size_t ws_bytes;
 };
@@ -85,7 +85,7 @@ int plan_group(bool tied, const void *q, const void *c0, const void *c1, const i
     if (!std::isfinite(scale)) return KVD_ERR_INVALID_ARG;
     if (h_q % h_kv) return KVD_ERR_INVALID_ARG;
     if (!q || !c0 || !c1 || !bt || !sl || !out || !lse) return KVD_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(c0, 16) || !aligned(c1, 16) || !aligned(out, 4) || !aligned(lse, 4) ||
+    if (!aligned(q, 16) || !aligned(c0, 16) || !aligned(c1, 16) || !aligned(out, 8) || !aligned(lse, 4) ||
         !aligned(bt, 4) || !aligned(sl, 4))
         return KVD_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return KVD_ERR_UNSUPPORTED_SHAPE;
@@ -103,8 +103,15 @@ int plan_group(bool tied, const void *q, const void *c0, const void *c1, const i
             gpc = g;
             break;
         }
-    const uint32_t kv_tile = (uint32_t)gpc * d * TILE * 2;
-    const uint32_t tx = tied ? kv_tile + TILE * d_r * 2 : 2 * kv_tile;
+    // 32-token stages (two independent MMA chains per wait) when a page holds whole 32-token
+    // tiles and at least three stages fit; otherwise 16-token stages.
+    auto stage_tx = [&](int tt) -> uint32_t {
+        const uint32_t kvt = (uint32_t)gpc * d * tt * 2;
+        return tied ? kvt + tt * d_r * 2 : 2 * kvt;
+    };
+    int tile = TILE;
+    if (nt == 1 && S % 32 == 0 && 3 * round_up(stage_tx(32), 1024) <= SMEM_BUDGET - 1024) tile = 32;
+    const uint32_t tx = stage_tx(tile);
     const uint32_t stage = (uint32_t)round_up(tx, 1024);
     int nstage = (int)((SMEM_BUDGET - 1024) / stage);
     if (nstage > MAX_STAGES) nstage = MAX_STAGES;
@@ -123,6 +130,7 @@ int plan_group(bool tied, const void *q, const void *c0, const void *c1, const i
     gp->parts = parts;
     gp->nt = nt;
     gp->nstage = nstage;
+    gp->tile = tile;
     gp->stage_bytes = stage;
     gp->stage_bytes_tx = tx;
     gp->ws_bytes = WS_HEADER + round_up(slots * rows * 4, 256) + slots * rows * d * 4;
@@ -145,14 +153,14 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
     {
         cuuint64_t dims[3] = {64, tokens, (cuuint64_t)h_kv * d / 64};
         cuuint64_t strides[2] = {(cuuint64_t)h_kv * d * 2, 128};
-        cuuint32_t box[3] = {64, (cuuint32_t)TILE, (cuuint32_t)(gp.gpc * d / 64)};
+        cuuint32_t box[3] = {64, (cuuint32_t)gp.tile, (cuuint32_t)(gp.gpc * d / 64)};
         if (!encode(&m0, c0, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
         if (!tied && !encode(&m1, c1, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
     }
     if (tied) {
         cuuint64_t dims[2] = {(cuuint64_t)d_r, tokens};
         cuuint64_t strides[1] = {(cuuint64_t)d_r * 2};
-        cuuint32_t box[2] = {(cuuint32_t)d_r, (cuuint32_t)TILE};
+        cuuint32_t box[2] = {(cuuint32_t)d_r, (cuuint32_t)gp.tile};
         if (!encode(&m1, c1, 2, dims, strides, box,
                     d_r == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
             return KVD_ERR_CUDA;
@@ -177,6 +185,7 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
     a.page_size = S;
     a.num_pages = P;
     a.max_pages = max_pages;
+    a.tile = gp.tile;
     a.gpc = gp.gpc;
     a.n_sub = gp.n_sub;
     a.parts = gp.parts;
@@ -200,7 +209,7 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
     c.lse = lse;
     c.B = B;
     c.L = L;
-    c.tile = TILE;
+    c.tile = gp.tile;
     c.max_tokens = max_pages * S;
     c.parts = gp.parts;
     c.rows = (int)rows;
@@ -209,9 +218,155 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
     return KVD_OK;
 }
 
+// ----------------------------------------------------------------------------- GLA / MLA
+// Shared memory a block may hold in total on sm_100 (227 KB).
+constexpr size_t SMEM_PER_BLOCK = 232448;
+// Static shared memory of the latent kernel is below this.
+constexpr size_t LATENT_STATIC_SMEM = 2048;
+
+struct LatentPlan {
+    LatentShape shape;
+    int n_rt, n_vc, n_sub, parts, nstage, rb;
+    size_t smem, ws_bytes;
+};
+
+int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
+    if (p->B < 0 || p->L < 1 || p->h_q < 1 || p->h_c < 1 || p->page_size < 1 || p->num_pages < 1 ||
+        p->max_pages < 1 || p->num_parts < 0)
+        return KVD_ERR_INVALID_ARG;
+    if (!std::isfinite(p->scale) || p->h_q % p->h_c) return KVD_ERR_INVALID_ARG;
+    if (!p->q || !p->latent_cache || !p->rope_cache || !p->block_table || !p->seqlens || !p->out || !p->lse)
+        return KVD_ERR_INVALID_ARG;
+    if (!aligned(p->q, 16) || !aligned(p->latent_cache, 16) || !aligned(p->rope_cache, 16) || !aligned(p->out, 16) ||
+        !aligned(p->lse, 4) || !aligned(p->block_table, 4) || !aligned(p->seqlens, 4))
+        return KVD_ERR_INVALID_ARG;
+    if (p->d_r != 64) return KVD_ERR_UNSUPPORTED_SHAPE;
+    LatentShape sh = latent_shape(p->d_c);
+    if (sh.tok == 0) return KVD_ERR_UNSUPPORTED_SHAPE;
+    if (p->page_size % sh.tok) return KVD_ERR_UNSUPPORTED_SHAPE;
+    const int g = p->h_q / p->h_c;
+    if (!(128 % g == 0 || g % 128 == 0)) return KVD_ERR_UNSUPPORTED_SHAPE;
+    const long long R = (long long)g * p->L;
+    if ((long long)p->num_pages * p->page_size >= (1ll << 31) || (long long)p->max_pages * p->page_size >= (1ll << 31) ||
+        (long long)p->B * p->L * p->h_q >= (1ll << 31) || R > 128 * 64)
+        return KVD_ERR_UNSUPPORTED_SHAPE;
+    lp->shape = sh;
+    lp->n_rt = (int)((R + 127) / 128);
+    lp->n_vc = p->d_c / 256;
+    lp->n_sub = p->h_c * lp->n_rt * lp->n_vc;
+    lp->rb = g < 128 ? g : 128;
+    const size_t fixed = SMEM_PER_BLOCK - LATENT_STATIC_SMEM - 1024 - sh.q_bytes - sh.p_bytes;
+    int nstage = (int)(fixed / sh.stage_bytes);
+    if (nstage > MAX_STAGES) nstage = MAX_STAGES;
+    if (nstage < 2) return KVD_ERR_UNSUPPORTED_SHAPE;
+    lp->nstage = nstage;
+    lp->smem = 1024 + sh.q_bytes + (size_t)nstage * sh.stage_bytes + sh.p_bytes;
+    int parts = p->num_parts;
+    if (parts == 0) {
+        const int sms = num_sms_current();
+        if (sms <= 0) return KVD_ERR_CUDA;
+        parts = sms / lp->n_sub > 0 ? sms / lp->n_sub : 1;
+    }
+    lp->parts = parts;
+    const size_t slots = (size_t)p->B + parts - 1;
+    const size_t rows = (size_t)p->L * p->h_q;
+    lp->ws_bytes = WS_HEADER + round_up(slots * rows * 4, 256) + slots * rows * p->d_c * 4;
+    return KVD_OK;
+}
+
+int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t st) {
+    LatentPlan lp;
+    int rc = plan_latent(p, &lp);
+    if (rc != KVD_OK) return rc;
+    if (!ws || !aligned(ws, 256)) return KVD_ERR_INVALID_ARG;
+    if (ws_bytes < lp.ws_bytes) return KVD_ERR_WORKSPACE_TOO_SMALL;
+    if (p->B == 0) return KVD_OK;
+
+    const int d_qk = p->d_c + p->d_r;
+    const int kch = d_qk / 64;
+    const cuuint64_t tokens = (cuuint64_t)p->num_pages * p->page_size;
+    CUtensorMap qm, lm, rm;
+    {
+        cuuint64_t dims[3] = {64, (cuuint64_t)p->B * p->L * p->h_q, (cuuint64_t)kch};
+        cuuint64_t strides[2] = {(cuuint64_t)d_qk * 2, 128};
+        cuuint32_t box[3] = {64, (cuuint32_t)lp.rb, 1};
+        if (!encode(&qm, p->q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[3] = {64, tokens, (cuuint64_t)p->h_c * p->d_c / 64};
+        cuuint64_t strides[2] = {(cuuint64_t)p->h_c * p->d_c * 2, 128};
+        cuuint32_t box[3] = {64, (cuuint32_t)lp.shape.tok, (cuuint32_t)(p->d_c / 64)};
+        if (!encode(&lm, p->latent_cache, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+    }
+    {
+        cuuint64_t dims[2] = {64, tokens};
+        cuuint64_t strides[1] = {128};
+        cuuint32_t box[2] = {64, (cuuint32_t)lp.shape.tok};
+        if (!encode(&rm, p->rope_cache, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+    }
+    const size_t slots = (size_t)p->B + lp.parts - 1;
+    const size_t rows = (size_t)p->L * p->h_q;
+    uint8_t *w = (uint8_t *)ws;
+    LatentArgs a;
+    a.q = (const __nv_bfloat16 *)p->q;
+    a.block_table = p->block_table;
+    a.seqlens = p->seqlens;
+    a.out = (__nv_bfloat16 *)p->out;
+    a.lse = p->lse;
+    a.err = (uint32_t *)w;
+    a.ws_lse = (float *)(w + WS_HEADER);
+    a.ws_o = (float *)(w + WS_HEADER + round_up(slots * rows * 4, 256));
+    a.B = p->B;
+    a.L = p->L;
+    a.h_q = p->h_q;
+    a.h_c = p->h_c;
+    a.page_size = p->page_size;
+    a.num_pages = p->num_pages;
+    a.max_pages = p->max_pages;
+    a.n_sub = lp.n_sub;
+    a.n_rt = lp.n_rt;
+    a.parts = lp.parts;
+    a.nstage = lp.nstage;
+    a.scale_log2 = p->scale * 1.4426950408889634f;
+    a.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
+    a.debug_flags = g_debug_flags.load();
+    record(g_ev_before, st);
+    if (launch_latent_decode(p->d_c, qm, lm, rm, a, lp.parts * lp.n_sub, lp.smem, st) != cudaSuccess)
+        return KVD_ERR_CUDA;
+    record(g_ev_after, st);
+
+    CombineArgs c;
+    c.seqlens = p->seqlens;
+    c.ws_lse = a.ws_lse;
+    c.ws_o = a.ws_o;
+    c.out = (__nv_bfloat16 *)p->out;
+    c.lse = p->lse;
+    c.B = p->B;
+    c.L = p->L;
+    c.tile = lp.shape.tok;
+    c.max_tokens = p->max_pages * p->page_size;
+    c.parts = lp.parts;
+    c.rows = (int)rows;
+    c.d_v = p->d_c;
+    if (launch_combine(c, st) != cudaSuccess) return KVD_ERR_CUDA;
+    return KVD_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t kvd_gla_workspace_size(const kvd_gla_params *p) {
+    if (!p) return 0;
+    LatentPlan lp;
+    if (plan_latent(p, &lp) != KVD_OK) return 0;
+    return lp.ws_bytes;
+}
+
+int kvd_gla_decode(const kvd_gla_params *p, void *ws, size_t ws_bytes, kvd_stream_t stream) {
+    if (!p) return KVD_ERR_INVALID_ARG;
+    return run_latent(p, ws, ws_bytes, (cudaStream_t)stream);
+}
 
 size_t kvd_gqa_workspace_size(const kvd_gqa_params *p) {
     if (!p) return 0;

@@ -90,19 +90,30 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     }
     __syncthreads();
 
-    const int dv = a.d_v;
-    for (int idx = threadIdx.x; idx < nrow * dv; idx += blockDim.x) {
-        const int w = idx / dv, col = idx % dv;
+    // out = sum_s w_s O_s: four consecutive columns per thread, the loads of all splits
+    // independent of each other so that they are in flight together
+    const int dv4 = a.d_v / 4;
+    for (int idx = threadIdx.x; idx < nrow * dv4; idx += blockDim.x) {
+        const int w = idx / dv4, c4 = idx % dv4;
         const int r = row0 + w;
         const float L = lse_sh[w];
-        float acc = 0.f;
+        const float4 *src = (const float4 *)(a.ws_o + ((size_t)(b + first) * rows + r) * a.d_v) + c4;
+        const size_t step4 = rows * a.d_v / 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
         for (int s = 0; s < nsplit; ++s) {
-            const size_t slot = (size_t)(b + first + s);
             const float wt = s < MAXW ? w_sh[w][s]
-                                      : (L == -INFINITY ? 0.f : expf(a.ws_lse[slot * rows + r] - L));
-            if (wt != 0.f) acc += wt * a.ws_o[(slot * rows + r) * dv + col];
+                                      : (L == -INFINITY ? 0.f : expf(a.ws_lse[(size_t)(b + first + s) * rows + r] - L));
+            const float4 x = __ldcs(src + (size_t)s * step4);
+            acc.x += wt * x.x;
+            acc.y += wt * x.y;
+            acc.z += wt * x.z;
+            acc.w += wt * x.w;
         }
-        a.out[((size_t)b * rows + r) * dv + col] = __float2bfloat16_rn(acc);
+        uint2 o;
+        o.x = pack_bf16(acc.x, acc.y);
+        o.y = pack_bf16(acc.z, acc.w);
+        *(uint2 *)(a.out + ((size_t)b * rows + r) * a.d_v + 4 * c4) = o;
     }
 }
 

@@ -30,7 +30,7 @@ namespace {
 
 constexpr int MAXSEG = 128;
 
-template <bool TIED, int D, int DR, int NT>
+template <bool TIED, int D, int DR, int NT, int TT>
 __global__ void __launch_bounds__(9 * 32, 1)
     group_decode_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
                         const GroupArgs a) {
@@ -48,7 +48,8 @@ __global__ void __launch_bounds__(9 * 32, 1)
     const int g_q = a.h_q / a.h_kv;
     const int R = g_q * a.L;
     const int max_tokens = a.max_pages * a.page_size;
-    const uint32_t kv_tile = (uint32_t)(gpc * D * TILE * 2);  // bytes of one K / V / tied tile
+    constexpr int NH = TT / 16;                                // 16-token MMA blocks per stage
+    const uint32_t kv_tile = (uint32_t)(gpc * D * TT * 2);    // bytes of one K / V / tied tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nstage; ++s) {
@@ -69,7 +70,7 @@ __global__ void __launch_bounds__(9 * 32, 1)
     for (int skip = 0;; skip += MAXSEG) {
         if (warp == gpc) {
             int cnt = 0;
-            plan_walk(a.seqlens, a.B, TILE, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
+            plan_walk(a.seqlens, a.B, TT, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
                 if (cnt >= skip && cnt < skip + MAXSEG) segs[cnt - skip] = s;
                 ++cnt;
             });
@@ -90,7 +91,7 @@ __global__ void __launch_bounds__(9 * 32, 1)
             for (int si = 0; si < nseg && !stop; ++si) {
                 const Seg sg = segs[si];
                 const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
-                const int tiles_per_page = a.page_size / TILE;
+                const int tiles_per_page = a.page_size / TT;
                 const int p_first = sg.t0 / tiles_per_page;
                 const int p_last = (sg.t1 - 1) / tiles_per_page;
                 for (int pb = p_first; pb <= p_last && !stop; pb += 32) {
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(9 * 32, 1)
                         }
                         if (lane == 0) {
                             uint8_t *st = smem + (size_t)stage * a.stage_bytes;
-                            const int row = pg * a.page_size + (t % tiles_per_page) * TILE;
+                            const int row = pg * a.page_size + (t % tiles_per_page) * TT;
                             mbar_arrive_expect_tx(&full_bar[stage], a.stage_bytes_tx);
                             if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || issued != 0) {
                                 tma_load_3d(st, &map0, &full_bar[stage], 0, row, z0, pol);
@@ -143,6 +144,30 @@ __global__ void __launch_bounds__(9 * 32, 1)
             const int gl = warp;                      // local group
             const int g = sub * gpc + gl;             // KV group
             const int lr = lane >> 2, lc = lane & 3;  // fragment row / column-pair
+            // Stage-relative shared-memory addresses of this lane's ldmatrix rows (the swizzle
+            // depends only on the lane).  koff: K (x4: tokens 8*(mi&1).., dims 8*(mi>>1)..);
+            // voff: V^T (x4.trans: dims 8*(mi&1).., tokens 8*(mi>>1)..).  The next 16 tokens sit
+            // 16 rows further on: +2048 bytes in 128-byte rows, +1024 in the 64-byte rope rows.
+            uint32_t koff[D / 16], khalf[D / 16], voff[D / 16];
+            {
+                const int mi = lane >> 3;
+                const int tk_k = (lane & 7) + 8 * (mi & 1);
+                const int tk_v = (lane & 7) + 8 * (mi >> 1);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int dim = kk * 16 + 8 * (mi >> 1);
+                    if (!TIED || kk * 16 < D - DR) {
+                        koff[kk] = sw128((gl * (D / 64) + dim / 64) * TT + tk_k, (dim & 63) >> 3);
+                        khalf[kk] = 2048;
+                    } else {
+                        const int rd = dim - (D - DR);
+                        koff[kk] = kv_tile + (DR == 64 ? sw128(tk_k, rd >> 3) : sw64(tk_k, rd >> 3));
+                        khalf[kk] = DR == 64 ? 2048 : 1024;
+                    }
+                    const int vdim = kk * 16 + 8 * (mi & 1);
+                    voff[kk] = (TIED ? 0u : kv_tile) + sw128((gl * (D / 64) + vdim / 64) * TT + tk_v, (vdim & 63) >> 3);
+                }
+            }
             for (int si = 0; si < nseg; ++si) {
                 const Seg sg = segs[si];
                 const int b = sg.b;
@@ -177,14 +202,23 @@ __global__ void __launch_bounds__(9 * 32, 1)
                         lim[nt][j] = n < R ? T - a.L + n / g_q : -1;
                     }
 
-                float m[NT][2], l[NT][2], o[NT][D / 16][4];
+                // m holds the reference maximum of each row (base 2, scale folded in).  It is
+                // only raised when a score exceeds it by more than 2^8, so P stays <= 256 and
+                // O is rescaled rarely.
+                // l: sum of the fp32 P (gives lse); lr: sum of the bf16-rounded P the product
+                // uses (normalises O, so the output is a convex combination of the rounded
+                // weights and a dominant token comes out exactly).
+                float m[NT][2], l[NT][2], lq[NT][2], o[NT][D / 16][4];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     m[nt][0] = m[nt][1] = -INFINITY;
                     l[nt][0] = l[nt][1] = 0.f;
+                    lq[nt][0] = lq[nt][1] = 0.f;
 #pragma unroll
                     for (int mt = 0; mt < D / 16; ++mt) o[nt][mt][0] = o[nt][mt][1] = o[nt][mt][2] = o[nt][mt][3] = 0.f;
                 }
+                // smallest causal limit over the real rows: tiles entirely at or below it need no mask
+                const int lim_all = T - a.L;
 
                 bool ok = true;
                 for (int tile = sg.t0; tile < sg.t1; ++tile, ++it) {
@@ -194,65 +228,74 @@ __global__ void __launch_bounds__(9 * 32, 1)
                         break;
                     }
                     const uint32_t base = smem_u32(smem + (size_t)stage * a.stage_bytes);
-                    const int tok0 = tile * TILE;
+                    const int tok0 = tile * TT;
 
-                    // ---- S^T = K q^T (tokens x rows)
-                    float s[NT][4];
+                    // ---- S^T = K q^T (tokens x rows), NH independent 16-token blocks
+                    float s[NH][NT][4];
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-                    {
-                        const int mi = lane >> 3;
-                        const int tk = (lane & 7) + 8 * (mi & 1);
+                    for (int h = 0; h < NH; ++h)
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const int dim = kk * 16 + 8 * (mi >> 1);
-                            uint32_t addr;
-                            if (!TIED || kk * 16 < D - DR) {
-                                const int row = (gl * (D / 64) + dim / 64) * TILE + tk;
-                                addr = base + sw128(row, (dim & 63) >> 3);
-                            } else {
-                                const int rd = dim - (D - DR);
-                                addr = base + kv_tile + (DR == 64 ? sw128(tk, rd >> 3) : sw64(tk, rd >> 3));
-                            }
+                        for (int nt = 0; nt < NT; ++nt) s[h][nt][0] = s[h][nt][1] = s[h][nt][2] = s[h][nt][3] = 0.f;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) {
                             uint32_t A[4];
-                            ldsm_x4(addr, A);
+                            ldsm_x4(base + koff[kk] + h * khalf[kk], A);
 #pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) mma_bf16(s[nt], A, qf[nt][kk][0], qf[nt][kk][1]);
+                            for (int nt = 0; nt < NT; ++nt) mma_bf16(s[h][nt], A, qf[nt][kk][0], qf[nt][kk][1]);
                         }
                     }
 
-                    // ---- mask, online softmax (base 2)
-                    const int ta = tok0 + lr, tb = ta + 8;
+                    // ---- mask (boundary tiles only), online softmax in base 2
+                    const bool full = tok0 + TT - 1 <= lim_all;
+#pragma unroll
+                    for (int h = 0; h < NH; ++h)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int t = tok0 + 16 * h + lr + 8 * (e >> 1);
+                                const float v = s[h][nt][e] * a.scale_log2;
+                                s[h][nt][e] = (full || t <= lim[nt][e & 1]) ? v : -INFINITY;
+                            }
                     float alpha[NT][2];
                     bool rescale = false;
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                         for (int j = 0; j < 2; ++j) {
-                            float v0 = ta <= lim[nt][j] ? s[nt][j] * a.scale_log2 : -INFINITY;
-                            float v1 = tb <= lim[nt][j] ? s[nt][2 + j] * a.scale_log2 : -INFINITY;
-                            float mx = fmaxf(v0, v1);
+                            float mx = -INFINITY;
+#pragma unroll
+                            for (int h = 0; h < NH; ++h) mx = fmaxf(mx, fmaxf(s[h][nt][j], s[h][nt][2 + j]));
                             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                            const float m_new = fmaxf(m[nt][j], mx);
-                            // nothing visible yet: O and l are still 0, leave them alone
-                            float al = 1.f, p0 = 0.f, p1 = 0.f;
-                            if (m_new != -INFINITY) {
-                                al = ex2(m[nt][j] - m_new);
-                                p0 = ex2(v0 - m_new);
-                                p1 = ex2(v1 - m_new);
+                            float al = 1.f;
+                            if (mx != -INFINITY) {
+                                if (m[nt][j] == -INFINITY) {
+                                    m[nt][j] = mx;  // first visible score: O and l still hold zeros
+                                } else if (mx > m[nt][j] + 8.f) {
+                                    al = ex2(m[nt][j] - mx);
+                                    m[nt][j] = mx;
+                                }
                             }
-                            m[nt][j] = m_new;
-                            l[nt][j] = l[nt][j] * al + p0 + p1;
-                            s[nt][j] = p0;
-                            s[nt][2 + j] = p1;
                             alpha[nt][j] = al;
                             rescale |= (al != 1.f);
+                            const float mr = m[nt][j] == -INFINITY ? 0.f : m[nt][j];
+#pragma unroll
+                            for (int h = 0; h < NH; ++h) {
+                                s[h][nt][j] = ex2(s[h][nt][j] - mr);
+                                s[h][nt][2 + j] = ex2(s[h][nt][2 + j] - mr);
+                            }
                         }
                     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt)
+                        for (int nt = 0; nt < NT; ++nt) {
+                            l[nt][0] *= alpha[nt][0];
+                            l[nt][1] *= alpha[nt][1];
+                            lq[nt][0] *= alpha[nt][0];
+                            lq[nt][1] *= alpha[nt][1];
 #pragma unroll
                             for (int mt = 0; mt < D / 16; ++mt) {
                                 o[nt][mt][0] *= alpha[nt][0];
@@ -260,42 +303,51 @@ __global__ void __launch_bounds__(9 * 32, 1)
                                 o[nt][mt][2] *= alpha[nt][0];
                                 o[nt][mt][3] *= alpha[nt][1];
                             }
-                    }
-
-                    // ---- P^T as B fragments (tokens x rows), via an 8x8 transpose per half
-                    uint32_t pb[NT][2];
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        pb[nt][0] = movmatrix_t(pack_bf16(s[nt][0], s[nt][1]));
-                        pb[nt][1] = movmatrix_t(pack_bf16(s[nt][2], s[nt][3]));
-                    }
-
-                    // ---- O^T += V^T P^T; tokens past T_b hold garbage (NaN poison): zero them
-                    const bool tail = tok0 + TILE > T;
-                    uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-                    if (tail) {
-                        const int t0 = tok0 + 2 * lc;
-                        mlo = (t0 < T ? 0x0000ffffu : 0u) | (t0 + 1 < T ? 0xffff0000u : 0u);
-                        mhi = (t0 + 8 < T ? 0x0000ffffu : 0u) | (t0 + 9 < T ? 0xffff0000u : 0u);
-                    }
-                    {
-                        const int mi = lane >> 3;
-                        const int tk = (lane & 7) + 8 * (mi >> 1);
-                        const uint32_t vbase = TIED ? base : base + kv_tile;
-#pragma unroll
-                        for (int mt = 0; mt < D / 16; ++mt) {
-                            const int dim = mt * 16 + 8 * (mi & 1);
-                            const int row = (gl * (D / 64) + dim / 64) * TILE + tk;
-                            uint32_t A[4];
-                            ldsm_x4_t(vbase + sw128(row, (dim & 63) >> 3), A);
-                            A[0] &= mlo;
-                            A[1] &= mlo;
-                            A[2] &= mhi;
-                            A[3] &= mhi;
-#pragma unroll
-                            for (int nt = 0; nt < NT; ++nt) mma_bf16(o[nt][mt], A, pb[nt][0], pb[nt][1]);
                         }
                     }
+
+                    // ---- P^T as B fragments (tokens x rows) via 8x8 transposes.  The normaliser
+                    // sums the same bf16-rounded P the product uses.
+                    uint32_t pb[NH][NT][2];
+#pragma unroll
+                    for (int h = 0; h < NH; ++h)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const uint32_t x0 = pack_bf16(s[h][nt][0], s[h][nt][1]);
+                            const uint32_t x1 = pack_bf16(s[h][nt][2], s[h][nt][3]);
+                            // (after the rescale above: l and lq were scaled to the current m first)
+                            l[nt][0] += s[h][nt][0] + s[h][nt][2];
+                            l[nt][1] += s[h][nt][1] + s[h][nt][3];
+                            lq[nt][0] += bf16_lo(x0) + bf16_lo(x1);
+                            lq[nt][1] += bf16_hi(x0) + bf16_hi(x1);
+                            pb[h][nt][0] = movmatrix_t(x0);
+                            pb[h][nt][1] = movmatrix_t(x1);
+                        }
+
+                    // ---- O^T += V^T P^T; tokens past T_b hold garbage (NaN poison): zero them
+                    uint32_t mlo[NH], mhi[NH];
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        mlo[h] = mhi[h] = 0xffffffffu;
+                        const int t0 = tok0 + 16 * h + 2 * lc;
+                        if (tok0 + TT > T) {
+                            mlo[h] = (t0 < T ? 0x0000ffffu : 0u) | (t0 + 1 < T ? 0xffff0000u : 0u);
+                            mhi[h] = (t0 + 8 < T ? 0x0000ffffu : 0u) | (t0 + 9 < T ? 0xffff0000u : 0u);
+                        }
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+                        for (int h = 0; h < NH; ++h) {
+                            uint32_t A[4];
+                            ldsm_x4_t(base + voff[mt] + h * 2048, A);
+                            A[0] &= mlo[h];
+                            A[1] &= mlo[h];
+                            A[2] &= mhi[h];
+                            A[3] &= mhi[h];
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) mma_bf16(o[nt][mt], A, pb[h][nt][0], pb[h][nt][1]);
+                        }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty_bar[stage]);
                 }
@@ -309,11 +361,15 @@ __global__ void __launch_bounds__(9 * 32, 1)
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        float v = l[nt][j];
+                        float v = l[nt][j], w = lq[nt][j];
                         v += __shfl_xor_sync(0xffffffffu, v, 4);
+                        w += __shfl_xor_sync(0xffffffffu, w, 4);
                         v += __shfl_xor_sync(0xffffffffu, v, 8);
+                        w += __shfl_xor_sync(0xffffffffu, w, 8);
                         v += __shfl_xor_sync(0xffffffffu, v, 16);
+                        w += __shfl_xor_sync(0xffffffffu, w, 16);
                         l[nt][j] = v;
+                        lq[nt][j] = w;
                     }
                 const int rows_b = a.L * a.h_q;
 #pragma unroll
@@ -324,7 +380,7 @@ __global__ void __launch_bounds__(9 * 32, 1)
                         if (n >= R) continue;
                         const int i = n / g_q, head = g * g_q + n % g_q;
                         const float lv = l[nt][j];
-                        const float inv = lv > 0.f ? 1.f / lv : 0.f;
+                        const float inv = lq[nt][j] > 0.f ? 1.f / lq[nt][j] : 0.f;
                         const float lse_v = lv > 0.f ? (m[nt][j] + lg2(lv)) * 0.69314718055994530942f : -INFINITY;
                         const int r = i * a.h_q + head;
                         if (sg.nsplit == 1) {
@@ -353,10 +409,10 @@ __global__ void __launch_bounds__(9 * 32, 1)
     }
 }
 
-template <bool TIED, int D, int DR, int NT>
+template <bool TIED, int D, int DR, int NT, int TT>
 cudaError_t launch_t(const CUtensorMap &m0, const CUtensorMap &m1, const GroupArgs &a, int grid, size_t smem,
                      cudaStream_t st) {
-    auto k = group_decode_kernel<TIED, D, DR, NT>;
+    auto k = group_decode_kernel<TIED, D, DR, NT, TT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<grid, (a.gpc + 1) * 32, smem, st>>>(m0, m1, a);
@@ -366,10 +422,12 @@ cudaError_t launch_t(const CUtensorMap &m0, const CUtensorMap &m1, const GroupAr
 template <bool TIED, int D, int DR>
 cudaError_t launch_nt(int nt, const CUtensorMap &m0, const CUtensorMap &m1, const GroupArgs &a, int grid,
                       size_t smem, cudaStream_t st) {
+    if (a.tile == 32 && nt == 1) return launch_t<TIED, D, DR, 1, 32>(m0, m1, a, grid, smem, st);
+    if (a.tile != 16) return cudaErrorInvalidValue;
     switch (nt) {
-        case 1: return launch_t<TIED, D, DR, 1>(m0, m1, a, grid, smem, st);
-        case 2: return launch_t<TIED, D, DR, 2>(m0, m1, a, grid, smem, st);
-        case 4: return launch_t<TIED, D, DR, 4>(m0, m1, a, grid, smem, st);
+        case 1: return launch_t<TIED, D, DR, 1, 16>(m0, m1, a, grid, smem, st);
+        case 2: return launch_t<TIED, D, DR, 2, 16>(m0, m1, a, grid, smem, st);
+        case 4: return launch_t<TIED, D, DR, 4, 16>(m0, m1, a, grid, smem, st);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -24,6 +24,7 @@ struct GroupArgs {
     float *ws_o;    // [slots][L * h_q][d]
     uint32_t *err;
     int B, L, h_q, h_kv, page_size, num_pages, max_pages;
+    int tile;   // tokens per pipeline stage (16 or 32)
     int gpc;    // KV groups per CTA (consumer warps)
     int n_sub;  // CTAs per part = h_kv / gpc
     int parts;
@@ -37,6 +38,37 @@ struct GroupArgs {
 
 cudaError_t launch_group_decode(bool tied, int d, int d_r, int nt, const CUtensorMap &m0, const CUtensorMap &m1,
                                 const GroupArgs &a, int grid, size_t smem, cudaStream_t st);
+
+struct LatentArgs {
+    const __nv_bfloat16 *q;
+    const int32_t *block_table;
+    const int32_t *seqlens;
+    __nv_bfloat16 *out;
+    float *lse;
+    float *ws_lse;  // [slots][L * h_q]
+    float *ws_o;    // [slots][L * h_q][d_c]
+    uint32_t *err;
+    int B, L, h_q, h_c, page_size, num_pages, max_pages;
+    int n_sub;  // CTAs per part = h_c * row blocks * value slices
+    int n_rt;   // 128-row blocks per latent head
+    int parts;
+    int nstage;
+    float scale_log2;
+    uint64_t wait_limit_ns;
+    int debug_flags;
+};
+
+// Compile-time geometry of the latent kernel for a latent width (0 fields: unsupported).
+struct LatentShape {
+    int tok;               // tokens per tile
+    uint32_t q_bytes;      // shared memory for the q block
+    uint32_t stage_bytes;  // one KV tile
+    uint32_t p_bytes;      // the P block
+};
+LatentShape latent_shape(int d_c);
+
+cudaError_t launch_latent_decode(int d_c, const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
+                                 const LatentArgs &a, int grid, size_t smem, cudaStream_t st);
 
 struct CombineArgs {
     const int32_t *seqlens;

@@ -1,0 +1,492 @@
+// GLA / MLA decode (absorbed form) over a paged latent cache on 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory).
+//
+// "Hardware-Efficient Attention for Fast Decoding", section 3.3.2: h_c latent
+// heads of width d_c plus one shared RoPE key of width d_r; query head h attends
+// latent head c = h / (h_q / h_c) with key [latent_c ++ rope] and value latent_c.
+// MLA is h_c = 1, d_c = 512.  All h_q / h_c query heads of a latent head (times
+// q_len) share every loaded latent row, so the step is a real dense contraction
+// (MLA: ~2 h_q FLOPs per byte, near the B200 ridge; GLA-2: ~h_q).
+//
+// One CTA owns one contiguous part of the (sequence, TOK-token tile) stream, one
+// latent head c, one 128-row block of the (q position, head) rows and one
+// 256-wide slice of the value (MLA's 512 value columns are split over two
+// neighbouring CTAs, since a 128 x 512 fp32 accumulator alone fills all of tensor
+// memory).  Roles:
+//   warp 0      producer: q rows of the segment, then per tile one 3-D TMA for
+//               the latent rows and one for the rope rows (128 B swizzle), into an
+//               n-stage mbarrier ring; block-table entries a warp at a time.
+//   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM S buffers
+//               (M 128 rows, N TOK tokens, K d_c + d_r), then O += P V (N 256,
+//               K TOK, V read MN-major straight from the latent tile); completion
+//               reported with tcgen05.commit on mbarriers.
+//   warps 4..7  softmax: thread = row = TMEM lane; load its S row, mask, fp32
+//               online softmax in base 2 with a lazy rescale (O in TMEM is
+//               rescaled only when the running max grows by more than 2^8), write
+//               P (bf16 pairs) back into tensor memory, double-buffered, where the
+//               P.V product reads it as its A operand; epilogue out / lse or split
+//               partials.
+// Tensor memory (512 columns): O [0, 256), S buffers [256, 256 + 2 TOK), P buffers
+// after them (TOK / 2 columns each).
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvd {
+
+namespace {
+
+constexpr int LMAXSEG = 32;
+constexpr int DV = 256;  // value columns per CTA (fp32 accumulator columns in TMEM)
+constexpr float RESCALE_LOG2 = 8.f;
+
+template <int DC, int TOK>
+struct LatCfg {
+    static constexpr int KCH = (DC + 64) / 64;           // 64-wide K chunks: latent, then rope
+    static constexpr int NVC = DC / DV;                   // value slices
+    static constexpr uint32_t Q_BYTES = KCH * 128 * 128;  // 128 rows x 128 B per chunk
+    static constexpr uint32_t CHUNK = TOK * 128;          // one 64-dim chunk of a tile
+    static constexpr uint32_t STAGE = KCH * CHUNK;
+    static constexpr uint32_t S_COL = DV;                 // TMEM columns of the two S buffers
+    static constexpr uint32_t P_COL = DV + 2 * TOK;       // TMEM columns of the two P buffers
+    static constexpr uint32_t P_COLS = TOK / 2;           // bf16 pairs per row
+};
+
+template <int DC, int TOK>
+__global__ void __launch_bounds__(256, 1)
+    latent_decode_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap latmap,
+                         const __grid_constant__ CUtensorMap ropemap, const LatentArgs a) {
+    using C = LatCfg<DC, TOK>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
+    __shared__ uint64_t qfull_bar, qempty_bar, sfull_bar[2], sfree_bar[2], pfull_bar[2], pfree_bar[2], end_bar;
+    __shared__ Seg segs[LMAXSEG];
+    __shared__ int nseg_sh, more_sh;
+    __shared__ volatile int abort_sh;
+    __shared__ uint32_t tmem_sh;
+
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *q_s = smem;
+    uint8_t *stage_s = smem + C::Q_BYTES;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int part = blockIdx.x / a.n_sub, sub = blockIdx.x % a.n_sub;
+    const int vc = sub % C::NVC;
+    const int rt = (sub / C::NVC) % a.n_rt;
+    const int c = sub / (C::NVC * a.n_rt);
+    const int g = a.h_q / a.h_c;
+    const int R = g * a.L;
+    const int max_tokens = a.max_pages * a.page_size;
+    const int nstage = a.nstage;
+    const uint64_t lim_ns = a.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nstage; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&qfull_bar, 1);
+        mbar_init(&qempty_bar, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sfull_bar[s], 1);
+            mbar_init(&sfree_bar[s], 4);
+            mbar_init(&pfull_bar[s], 4);
+            mbar_init(&pfree_bar[s], 1);
+        }
+        mbar_init(&end_bar, 1);
+        abort_sh = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&tmem_sh, 512);
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&qmap);
+        tma_prefetch_desc(&latmap);
+        tma_prefetch_desc(&ropemap);
+    }
+    pdl_launch_dependents();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_sh;
+
+    // counters that persist across segment-list rounds
+    uint32_t p_issued = 0, p_qloads = 0;                    // producer
+    uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;        // MMA issuer
+    uint32_t x_tile = 0, x_s = 0, x_pv = 0;                 // softmax
+
+    for (int skip = 0;; skip += LMAXSEG) {
+        if (warp == 0) {
+            int cnt = 0;
+            plan_walk(a.seqlens, a.B, TOK, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
+                if (cnt >= skip && cnt < skip + LMAXSEG) segs[cnt - skip] = s;
+                ++cnt;
+            });
+            if (lane == 0) {
+                nseg_sh = cnt - skip < LMAXSEG ? (cnt - skip > 0 ? cnt - skip : 0) : LMAXSEG;
+                more_sh = cnt > skip + LMAXSEG;
+            }
+        }
+        __syncthreads();
+        const int nseg = nseg_sh;
+
+        if (warp == 0) {
+            // ================================================================ producer
+            const uint64_t pol = policy_evict_first();
+            bool stop = false;
+            const int rb = g < 128 ? g : 128;                      // q rows per TMA box
+            const int rows_tile = min(R - rt * 128, 128);          // valid rows of this row block
+            for (int si = 0; si < nseg && !stop; ++si) {
+                const Seg sg = segs[si];
+                if (!mbar_wait_warp(&qempty_bar, (p_qloads & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&qfull_bar, (uint32_t)rows_tile * C::KCH * 128);
+                    for (int run = 0; run * rb < rows_tile; ++run) {
+                        const int n0 = rt * 128 + run * rb;
+                        const int i = n0 / g, h0 = n0 % g;
+                        const int row = (sg.b * a.L + i) * a.h_q + c * g + h0;
+                        for (int ch = 0; ch < C::KCH; ++ch)
+                            tma_load_3d(q_s + ch * 16384 + run * rb * 128, &qmap, &qfull_bar, 0, row, ch, pol);
+                    }
+                }
+                ++p_qloads;
+                const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
+                const int tpp = a.page_size / TOK;
+                const int p_first = sg.t0 / tpp, p_last = (sg.t1 - 1) / tpp;
+                for (int pb = p_first; pb <= p_last && !stop; pb += 32) {
+                    int page = 0;
+                    if (pb + lane <= p_last) {
+                        page = __ldg(bt + pb + lane);
+                        if (page < 0 || page >= a.num_pages) {
+                            set_error(a.err, DEVERR_BAD_PAGE);
+                            page = 0;
+                        }
+                    }
+                    const int t_lo = max(sg.t0, pb * tpp), t_hi = min(sg.t1, (pb + 32) * tpp);
+                    for (int t = t_lo; t < t_hi; ++t) {
+                        const int pg = __shfl_sync(0xffffffffu, page, t / tpp - pb);
+                        const uint32_t stage = p_issued % nstage;
+                        if (!mbar_wait_warp(&empty_bar[stage], ((p_issued / nstage) & 1) ^ 1, &abort_sh, a.err,
+                                            lim_ns)) {
+                            stop = true;
+                            break;
+                        }
+                        if (lane == 0) {
+                            uint8_t *st = stage_s + (size_t)stage * C::STAGE;
+                            const int row = pg * a.page_size + (t % tpp) * TOK;
+                            mbar_arrive_expect_tx(&full_bar[stage], C::STAGE);
+                            if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0) {
+                                tma_load_3d(st, &latmap, &full_bar[stage], 0, row, c * (DC / 64), pol);
+                                tma_load_2d(st + (DC / 64) * C::CHUNK, &ropemap, &full_bar[stage], 0, row, pol);
+                            }
+                        }
+                        ++p_issued;
+                    }
+                }
+            }
+            if (stop) {
+                volatile int never = 0;
+                const uint32_t lo = p_issued > (uint32_t)nstage ? p_issued - nstage : 0;
+                for (uint32_t k = lo; k < p_issued; ++k)
+                    mbar_wait_warp(&full_bar[k % nstage], (k / nstage) & 1, &never, nullptr, lim_ns);
+                if (p_qloads) mbar_wait_warp(&qfull_bar, (p_qloads - 1) & 1, &never, nullptr, lim_ns);
+            }
+        } else if (warp == 1) {
+            // ================================================================ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idesc_s = umma_idesc_bf16(128, TOK, false, false);
+                constexpr uint32_t idesc_pv = umma_idesc_bf16(128, DV, false, true);
+                const uint32_t q_addr = smem_u32(q_s), st0 = smem_u32(stage_s);
+                bool ok = true;
+                auto issue_s = [&](uint32_t gt) -> bool {
+                    const uint32_t stage = gt % nstage;
+                    if (!mbar_wait_one(&full_bar[stage], (gt / nstage) & 1, &abort_sh, a.err, lim_ns)) return false;
+                    const uint32_t sb = m_s & 1;
+                    if (!mbar_wait_one(&sfree_bar[sb], ((m_s >> 1) & 1) ^ 1, &abort_sh, a.err, lim_ns)) return false;
+                    tc_fence_after();
+                    const uint32_t d = tmem + C::S_COL + sb * TOK;
+                    const uint32_t kv = st0 + stage * C::STAGE;
+#pragma unroll 1
+                    for (int kc = 0; kc < C::KCH; ++kc)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t da = umma_desc(q_addr + kc * 16384 + kk * 32, 16, 1024, 2);
+                            const uint64_t db = umma_desc(kv + kc * C::CHUNK + kk * 32, 16, 1024, 2);
+                            umma_bf16(d, da, db, idesc_s, (kc | kk) != 0);
+                        }
+                    umma_commit(&sfull_bar[sb]);
+                    ++m_s;
+                    return true;
+                };
+                for (int si = 0; si < nseg && ok; ++si) {
+                    const int n = segs[si].t1 - segs[si].t0;
+                    if (!mbar_wait_one(&qfull_bar, m_q & 1, &abort_sh, a.err, lim_ns)) break;
+                    ++m_q;
+                    tc_fence_after();
+                    if (!issue_s(m_tile)) break;
+                    if (n == 1) umma_commit(&qempty_bar);
+                    for (int j = 0; j < n; ++j) {
+                        if (j + 1 < n) {
+                            if (!issue_s(m_tile + j + 1)) {
+                                ok = false;
+                                break;
+                            }
+                            if (j + 1 == n - 1) umma_commit(&qempty_bar);
+                        }
+                        const uint32_t pb = m_pv & 1;
+                        if (!mbar_wait_one(&pfull_bar[pb], (m_pv >> 1) & 1, &abort_sh, a.err, lim_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t stage = (m_tile + j) % nstage;
+                        const uint32_t v0 = st0 + stage * C::STAGE + vc * 4 * C::CHUNK;
+                        const uint32_t pa = tmem + C::P_COL + pb * C::P_COLS;
+#pragma unroll
+                        for (int kk = 0; kk < TOK / 16; ++kk) {
+                            const uint64_t db = umma_desc(v0 + kk * 2048, C::CHUNK, 1024, 2);
+                            umma_bf16_ts(tmem, pa + kk * 8, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&pfree_bar[pb]);
+                        umma_commit(&empty_bar[stage]);
+                        ++m_pv;
+                    }
+                    m_tile += n;
+                }
+            }
+            __syncwarp();
+        } else if (warp >= 4) {
+            // ================================================================ softmax / epilogue
+            const int r = threadIdx.x - 128;
+            const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+            const int n_row = rt * 128 + r;
+            const bool row_ok = n_row < R;
+            const int i_row = row_ok ? n_row / g : 0;
+            const int head = row_ok ? c * g + n_row % g : 0;
+            bool ok = true;
+            // wait until P.V number k has completed (it frees P buffer k & 1 and settles O)
+            auto wait_pv = [&](uint32_t k) -> bool {
+                return mbar_wait_warp(&pfree_bar[k & 1], (k >> 1) & 1, &abort_sh, a.err, lim_ns);
+            };
+            for (int si = 0; si < nseg && ok; ++si) {
+                const Seg sg = segs[si];
+                const int b = sg.b;
+                const int T = clamp_len(__ldg(a.seqlens + b), max_tokens, a.L, nullptr);
+                const int lim = row_ok ? T - a.L + i_row : -1;
+                // l: sum of the fp32 P (gives lse); lq: sum of the bf16-rounded P the product
+                // uses (normalises O: a convex combination of the rounded weights).
+                float m_ref = -INFINITY, l = 0.f, lq = 0.f;
+                for (int tile = sg.t0; tile < sg.t1; ++tile) {
+                    const int tok0 = tile * TOK;
+                    const uint32_t sb = x_s & 1;
+                    if (!mbar_wait_warp(&sfull_bar[sb], (x_s >> 1) & 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    float s[TOK];
+                    {
+                        float tmp[32];
+                        tmem_ld32(tmem + lane_base + C::S_COL + sb * TOK, tmp);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) s[k] = tmp[k];
+                        if constexpr (TOK == 64) {
+                            tmem_ld32(tmem + lane_base + C::S_COL + sb * TOK + 32, tmp);
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) s[32 + k] = tmp[k];
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sfree_bar[sb]);
+                    ++x_s;
+
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < TOK; ++k) {
+                        const float v = (tok0 + k <= lim) ? s[k] * a.scale_log2 : -INFINITY;
+                        s[k] = v;
+                        mx = fmaxf(mx, v);
+                    }
+                    float alpha = 1.f;
+                    bool need = false;
+                    if (mx != -INFINITY) {
+                        if (m_ref == -INFINITY) {
+                            m_ref = mx;  // nothing visible before: O and l hold zeros
+                        } else if (mx > m_ref + RESCALE_LOG2) {
+                            alpha = ex2(m_ref - mx);
+                            need = true;
+                            m_ref = mx;
+                        }
+                    }
+                    if (__any_sync(0xffffffffu, need)) {
+                        // O is settled once the previous P.V (and so every earlier one) is done
+                        if (x_pv > 0 && !wait_pv(x_pv - 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        l *= alpha;
+                        lq *= alpha;
+#pragma unroll 1
+                        for (int ch = 0; ch < DV / 32; ++ch) {
+                            float o[32];
+                            tmem_ld32(tmem + lane_base + ch * 32, o);
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) o[k] *= alpha;
+                            tmem_st32(tmem + lane_base + ch * 32, o);
+                        }
+                        tmem_st_wait();
+                    }
+                    if (m_ref != -INFINITY) {
+#pragma unroll
+                        for (int k = 0; k < TOK; ++k) {
+                            s[k] = ex2(s[k] - m_ref);
+                            l += s[k];
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < TOK; ++k) s[k] = 0.f;
+                    }
+
+                    // tokens past T_b in this tile hold garbage: zero their value rows (P is 0 there,
+                    // but 0 * NaN would still poison the product)
+                    const uint32_t stage = x_tile % nstage;
+                    if (tok0 + TOK > T) {
+                        const int k0 = max(T - tok0, 0);
+                        uint8_t *v0 = stage_s + (size_t)stage * C::STAGE + (size_t)vc * 4 * C::CHUNK;
+                        const int units = (TOK - k0) * 4 * 8;  // 16-byte units: rows x 4 chunks x 8
+                        for (int u = r; u < units; u += 128) {
+                            const int row = k0 + u / 32, ch = (u / 8) & 3, k = u & 7;
+                            *(uint4 *)(v0 + ch * C::CHUNK + row * 128 + k * 16) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    // P row (bf16 pairs) -> tensor memory buffer x_pv & 1, once the P.V that last
+                    // read that buffer has completed.  The normaliser sums the same rounded values
+                    // the product uses.
+                    if (x_pv >= 2 && !wait_pv(x_pv - 2)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    float sum = 0.f;
+                    {
+                        const uint32_t pa = tmem + lane_base + C::P_COL + (x_pv & 1) * C::P_COLS;
+#pragma unroll
+                        for (int h = 0; h < TOK / 32; ++h) {
+                            uint32_t w[16];
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) {
+                                w[k] = pack_bf16(s[32 * h + 2 * k], s[32 * h + 2 * k + 1]);
+                                sum += bf16_lo(w[k]) + bf16_hi(w[k]);
+                            }
+                            tmem_st16u(pa + 16 * h, w);
+                        }
+                        tmem_st_wait();
+                    }
+                    lq += sum;
+                    if (tok0 + TOK > T) fence_proxy_async();  // the zeroed value rows above
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pfull_bar[x_pv & 1]);
+                    ++x_pv;
+                    ++x_tile;
+                }
+                if (!ok) break;
+
+                // ---- epilogue: O is final once the last P.V completes
+                if (!wait_pv(x_pv - 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float inv = lq > 0.f ? 1.f / lq : 0.f;
+                const float lse_v = l > 0.f ? (m_ref + lg2(l)) * 0.69314718055994530942f : -INFINITY;
+                const size_t rows_b = (size_t)a.L * a.h_q;
+                const size_t r_out = (size_t)i_row * a.h_q + head;
+#pragma unroll 1
+                for (int ch = 0; ch < DV / 32; ++ch) {
+                    float o[32];
+                    tmem_ld32(tmem + lane_base + ch * 32, o);
+                    if (!row_ok) continue;
+                    if (sg.nsplit == 1) {
+                        uint4 *op = (uint4 *)(a.out + ((size_t)b * rows_b + r_out) * DC + vc * DV + ch * 32);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            op[k] = make_uint4(pack_bf16(o[8 * k] * inv, o[8 * k + 1] * inv),
+                                               pack_bf16(o[8 * k + 2] * inv, o[8 * k + 3] * inv),
+                                               pack_bf16(o[8 * k + 4] * inv, o[8 * k + 5] * inv),
+                                               pack_bf16(o[8 * k + 6] * inv, o[8 * k + 7] * inv));
+                    } else {
+                        float4 *op = (float4 *)(a.ws_o + ((size_t)sg.slot * rows_b + r_out) * DC + vc * DV + ch * 32);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            op[k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv,
+                                                o[4 * k + 3] * inv);
+                    }
+                }
+                if (row_ok && vc == 0) {
+                    if (sg.nsplit == 1)
+                        a.lse[(size_t)b * rows_b + r_out] = lse_v;
+                    else
+                        a.ws_lse[(size_t)sg.slot * rows_b + r_out] = lse_v;
+                }
+                tc_fence_before();
+            }
+        }
+        __syncthreads();
+        if (!more_sh || abort_sh) break;
+        __syncthreads();
+    }
+
+    // every MMA issued by this CTA has completed before tensor memory is released
+    if (warp == 1 && lane == 0) {
+        volatile int never = 0;
+        umma_commit(&end_bar);
+        mbar_wait_one(&end_bar, 0, &never, nullptr, lim_ns);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int DC, int TOK>
+cudaError_t launch_t(const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a,
+                     int grid, size_t smem, cudaStream_t st) {
+    auto k = latent_decode_kernel<DC, TOK>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, 256, smem, st>>>(qm, lm, rm, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+LatentShape latent_shape(int d_c) {
+    LatentShape s{};
+    if (d_c == 256) {
+        s.tok = 64;
+        s.q_bytes = LatCfg<256, 64>::Q_BYTES;
+        s.stage_bytes = LatCfg<256, 64>::STAGE;
+        s.p_bytes = 0;
+    } else if (d_c == 512) {
+        s.tok = 32;
+        s.q_bytes = LatCfg<512, 32>::Q_BYTES;
+        s.stage_bytes = LatCfg<512, 32>::STAGE;
+        s.p_bytes = 0;
+    }
+    return s;
+}
+
+cudaError_t launch_latent_decode(int d_c, const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
+                                 const LatentArgs &a, int grid, size_t smem, cudaStream_t st) {
+    if (d_c == 256) return launch_t<256, 64>(qm, lm, rm, a, grid, smem, st);
+    if (d_c == 512) return launch_t<512, 32>(qm, lm, rm, a, grid, smem, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kvd

@@ -141,3 +141,33 @@ def test_plan_clamps_oversized_lengths():
     segs, counts = binding.plan_host(np.array([100, 5000], np.int32), 16, 256, 2)
     tiles = sum(int(segs[c, k, 2] - segs[c, k, 1]) for c in range(2) for k in range(counts[c]))
     assert tiles == 7 + 16
+
+
+def _gla_params(**kw):
+    base = dict(q=16, latent_cache=16, rope_cache=16, block_table=16, seqlens=16, out=16, lse=16,
+                B=2, L=1, h_q=128, h_c=2, d_c=256, d_r=64, page_size=64, num_pages=10, max_pages=8,
+                scale=0.07, num_parts=4)
+    base.update(kw)
+    return binding.GLAParams(**base)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(latent_cache=None), -1),
+    (dict(out=24), -1),                 # GLA output rows are written as 16-byte vectors
+    (dict(h_q=127), -1),
+    (dict(d_c=384), -2),                # latent width outside the compiled set
+    (dict(d_r=32), -2),
+    (dict(page_size=48), -2),           # not a multiple of the 64-token tile (d_c 256)
+    (dict(h_q=96, h_c=1), -2),          # 96 heads per latent head: neither divides nor is a multiple of 128
+])
+def test_gla_validation_errors(lib, kw, expect):
+    p = _gla_params(**kw)
+    assert lib.kvd_gla_workspace_size(ctypes.byref(p)) == 0
+    assert lib.kvd_gla_decode(ctypes.byref(p), ctypes.c_void_p(256), 1 << 30, None) == expect
+
+
+def test_gla_workspace_size(lib):
+    p = _gla_params(L=2, d_c=512, h_c=1, page_size=64)
+    n = lib.kvd_gla_workspace_size(ctypes.byref(p))
+    slots, rows = 2 + 4 - 1, 2 * 128
+    assert n == 256 + ((slots * rows * 4 + 255) // 256) * 256 + slots * rows * 512 * 4

@@ -1,0 +1,117 @@
+"""GLA / MLA (absorbed) decode on the GPU against the fp64 oracle (the benchmark spec tolerance)."""
+import numpy as np
+import pytest
+
+from kv_cache_paged_b200 import workload as wl
+from oracle import oracle as orc
+from tests import gpu_util as gu
+from tests.indexing import decode_digits, make_delta_problem
+
+pytestmark = pytest.mark.gpu
+
+
+def check(inp, num_parts=0, b_sample=None, what="", stress=True):
+    """Workload tests pass stress=False (plain the benchmark spec bound); the synthetic edge and
+    stress shapes use the magnitude-aware bound of gpu_util.assert_close."""
+    out, lse = gu.run_gpu(inp, num_parts=num_parts)
+    o, l = gu.to_np(out, lse)
+    if b_sample is not None:
+        sel = np.asarray(b_sample, dtype=np.int32)
+        ref_o, ref_l, _ = orc.decode_inputs(inp, b_list=sel)
+        return gu.assert_close(o[sel], l[sel], ref_o, ref_l, what or inp.name, stress=stress)
+    ref_o, ref_l, _ = orc.decode_inputs(inp)
+    return gu.assert_close(o, l, ref_o, ref_l, what or inp.name, stress=stress)
+
+
+def small(h_c, d_c, **kw):
+    base = dict(B=3, L=1, h_q=128, h_kv=h_c, d=d_c, d_r=64, page_size=64, seqlens=[1, 97, 300], seed=7,
+                scale=1.0 / np.sqrt(192), latent_scale=0.1 if h_c == 1 else 1.0)
+    base.update(kw)
+    return wl.make_inputs("gla", **base)
+
+
+# ----------------------------------------------------------------------------- small shapes first
+@pytest.mark.parametrize("L", [1, 2])
+def test_mla_small(cuda_device, L):
+    check(small(1, 512, L=L, seqlens=[L, 97, 300]), what=f"MLA L={L}")
+
+
+@pytest.mark.parametrize("L", [1, 2, 4])
+def test_gla2_small(cuda_device, L):
+    check(small(2, 256, L=L, seqlens=[L, 97, 300]), what=f"GLA-2 L={L}")
+
+
+@pytest.mark.parametrize("h_c,d_c", [(1, 512), (2, 256)])
+@pytest.mark.parametrize("num_parts", [1, 3, 50])
+def test_latent_forced_splits(cuda_device, h_c, d_c, num_parts):
+    inp = small(h_c, d_c, B=5, L=2, seqlens=("uniform", 2, 900), seed=11 + num_parts)
+    check(inp, num_parts=num_parts, what=f"h_c={h_c} parts={num_parts}")
+
+
+@pytest.mark.parametrize("h_c,d_c", [(1, 512), (2, 256)])
+def test_latent_page_boundaries(cuda_device, h_c, d_c):
+    sl = [1, 31, 32, 33, 63, 64, 65, 128, 129]
+    check(small(h_c, d_c, B=len(sl), seqlens=sl, seed=13), num_parts=4)
+
+
+@pytest.mark.parametrize("h_c,h_q,L", [(8, 128, 2), (4, 64, 1), (1, 64, 3), (2, 256, 1)])
+def test_latent_group_shapes(cuda_device, h_c, h_q, L):
+    """GLA-8 (16 heads per latent head), smaller and larger groups, q_len 3."""
+    inp = small(h_c, 256, h_q=h_q, L=L, seqlens=("uniform", L, 500), seed=h_c + h_q + L)
+    check(inp, what=f"h_c={h_c} h_q={h_q} L={L}")
+
+
+def test_latent_peaky_softmax(cuda_device):
+    inp = small(2, 256, L=2, seqlens=("uniform", 2, 2000), seed=17)
+    inp.scale *= 8
+    check(inp, num_parts=9)
+
+
+def test_latent_empty_sequences(cuda_device):
+    inp = small(2, 256, B=4, seqlens=[0, 70, 0, 5], seed=19)
+    out, lse = gu.run_gpu(inp, num_parts=3)
+    o, l = gu.to_np(out, lse)
+    assert np.all(o[[0, 2]] == 0) and np.all(np.isneginf(l[[0, 2]]))
+    ref_o, ref_l, _ = orc.decode_inputs(inp)
+    gu.assert_close(o, l, ref_o, ref_l, stress=True)
+
+
+# ----------------------------------------------------------------------------- indexing
+@pytest.mark.parametrize("h_c,d_c", [(1, 512), (2, 256)])
+def test_latent_delta_attention_exact_index(cuda_device, h_c, d_c):
+    inp, targets = make_delta_problem("gla", seed=23, B=4, h_q=32 * h_c, h_kv=h_c, d=d_c, d_r=64, S=64,
+                                      seqlens=("uniform", 20, 900))
+    out, lse = gu.run_gpu(inp, num_parts=5)
+    assert np.array_equal(decode_digits(inp, gu.to_np(out, lse)[0]), targets)
+
+
+def test_latent_page_permutation_bit_identical(cuda_device):
+    import torch
+    inp = small(2, 256, B=4, L=2, seqlens=("uniform", 2, 800), seed=29)
+    out1, lse1 = gu.run_gpu(inp)
+    perm = np.random.default_rng(0).permutation(inp.num_pages)
+    inv = np.argsort(perm)
+    for k in inp.caches:
+        inp.caches[k] = np.ascontiguousarray(inp.caches[k][inv])
+    bt = inp.block_table.copy()
+    bt[bt >= 0] = perm[bt[bt >= 0]]
+    inp.block_table = bt
+    out2, lse2 = gu.run_gpu(inp)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(lse1, lse2)
+
+
+# ----------------------------------------------------------------------------- full workloads (sampled)
+@pytest.mark.parametrize("L", [1, 2])
+def test_mla_workload_full_size(cuda_device, L):
+    """B 64, h_q 128, one 512-dim latent head + 64 rope, contexts U[4096, 32768]; 6 sequences checked."""
+    inp = wl.make_workload("mla", L=L)
+    check(inp, b_sample=[0, 7, 19, 33, 48, 63], what=f"MLA workload L={L}", stress=False)
+
+
+@pytest.mark.parametrize("L", [1, 2, 4])
+def test_gla2_workload_full_size(cuda_device, L):
+    """B 128, h_q 128 over two 256-dim latent heads + 64 rope, lognormal contexts; 6 sequences checked."""
+    inp = wl.make_workload("gla2", L=L)
+    longest = int(np.argmax(inp.seqlens))
+    check(inp, b_sample=[0, 5, 40, 77, 127, longest], what=f"GLA-2 workload L={L}", stress=False)
