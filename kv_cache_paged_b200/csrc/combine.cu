@@ -16,12 +16,9 @@ namespace kvd {
 
 namespace {
 
-constexpr int CROWS = 8;   // rows per CTA, one warp each for the lse step
-constexpr int MAXW = 64;   // weights cached in shared memory per row
+constexpr int CROWS = 8;   // rows per CTA
 
 __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
-    __shared__ float w_sh[CROWS][MAXW];
-    __shared__ float lse_sh[CROWS];
     __shared__ int first_sh, nsplit_sh;
 
     // Wait for the decode grid to finish and its partials to be visible.
@@ -69,51 +66,43 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     const int first = first_sh;
     const size_t rows = (size_t)a.rows;
 
-    if (warp < nrow) {
-        const int r = row0 + warp;
-        float m = -INFINITY;
-        for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, a.ws_lse[(size_t)(b + first + s) * rows + r]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float sum = 0.f;
-        if (m != -INFINITY)
-            for (int s = lane; s < nsplit; s += 32) sum += expf(a.ws_lse[(size_t)(b + first + s) * rows + r] - m);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        const float L = m == -INFINITY ? -INFINITY : m + logf(sum);
-        for (int s = lane; s < min(nsplit, MAXW); s += 32)
-            w_sh[warp][s] = L == -INFINITY ? 0.f : expf(a.ws_lse[(size_t)(b + first + s) * rows + r] - L);
-        if (lane == 0) {
-            lse_sh[warp] = L;
-            a.lse[(size_t)b * rows + r] = L;
-        }
-    }
-    __syncthreads();
-
-    // out = sum_s w_s O_s: four consecutive columns per thread, the loads of all splits
-    // independent of each other so that they are in flight together
+    // One memory round: each thread owns four consecutive outputs of one row and loads that
+    // row's lse and its four columns from every part together, then reduces locally.
     const int dv4 = a.d_v / 4;
     for (int idx = threadIdx.x; idx < nrow * dv4; idx += blockDim.x) {
-        const int w = idx / dv4, c4 = idx % dv4;
-        const int r = row0 + w;
-        const float L = lse_sh[w];
-        const float4 *src = (const float4 *)(a.ws_o + ((size_t)(b + first) * rows + r) * a.d_v) + c4;
-        const size_t step4 = rows * a.d_v / 4;
+        const int r = row0 + idx / dv4, c4 = idx % dv4;
+        float mx = -INFINITY, sum = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int s = 0; s < nsplit; ++s) {
-            const float wt = s < MAXW ? w_sh[w][s]
-                                      : (L == -INFINITY ? 0.f : expf(a.ws_lse[(size_t)(b + first + s) * rows + r] - L));
-            const float4 x = __ldcs(src + (size_t)s * step4);
-            acc.x += wt * x.x;
-            acc.y += wt * x.y;
-            acc.z += wt * x.z;
-            acc.w += wt * x.w;
+        for (int s0 = 0; s0 < nsplit; s0 += 8) {
+            float ls[8];
+            float4 x[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const size_t slot = (size_t)(b + first) + min(s0 + k, nsplit - 1);
+                ls[k] = s0 + k < nsplit ? __ldcs(a.ws_lse + slot * rows + r) : -INFINITY;
+                x[k] = __ldcs((const float4 *)(a.ws_o + (slot * rows + r) * a.d_v) + c4);
+            }
+            // streaming log-sum-exp over the parts, rescaling what is summed so far
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                if (ls[k] == -INFINITY) continue;
+                const float mn = fmaxf(mx, ls[k]);
+                const float sc = mx == -INFINITY ? 0.f : expf(mx - mn);
+                const float wk = expf(ls[k] - mn);
+                sum = sum * sc + wk;
+                acc.x = acc.x * sc + wk * x[k].x;
+                acc.y = acc.y * sc + wk * x[k].y;
+                acc.z = acc.z * sc + wk * x[k].z;
+                acc.w = acc.w * sc + wk * x[k].w;
+                mx = mn;
+            }
         }
+        const float inv = sum > 0.f ? 1.f / sum : 0.f;
         uint2 o;
-        o.x = pack_bf16(acc.x, acc.y);
-        o.y = pack_bf16(acc.z, acc.w);
+        o.x = pack_bf16(acc.x * inv, acc.y * inv);
+        o.y = pack_bf16(acc.z * inv, acc.w * inv);
         *(uint2 *)(a.out + ((size_t)b * rows + r) * a.d_v + 4 * c4) = o;
+        if (c4 == 0) a.lse[(size_t)b * rows + r] = mx == -INFINITY ? -INFINITY : mx + logf(sum);
     }
 }
 
