@@ -222,7 +222,7 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
 // Shared memory a block may hold in total on sm_100 (227 KB).
 constexpr size_t SMEM_PER_BLOCK = 232448;
 // Static shared memory of the latent kernel is below this.
-constexpr size_t LATENT_STATIC_SMEM = 2048;
+constexpr size_t LATENT_STATIC_SMEM = 4096;
 
 struct LatentPlan {
     LatentShape shape;

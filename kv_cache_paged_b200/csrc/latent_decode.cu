@@ -20,7 +20,8 @@
 //               (M 128 rows, N TOK tokens, K d_c + d_r), then O += P V (N 256,
 //               K TOK, V read MN-major straight from the latent tile); completion
 //               reported with tcgen05.commit on mbarriers.
-//   warps 4..7  softmax: thread = row = TMEM lane; load its S row, mask, fp32
+//   warps 4..11 softmax: a row (TMEM lane) is shared by two threads, one per column half
+//               of the tile; each loads its half of the S row, masks, runs the fp32
 //               online softmax in base 2 with a lazy rescale (O in TMEM is
 //               rescaled only when the running max grows by more than 2^8), write
 //               P (bf16 pairs) back into tensor memory, double-buffered, where the
@@ -54,7 +55,7 @@ struct LatCfg {
 };
 
 template <int DC, int TOK>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     latent_decode_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap latmap,
                          const __grid_constant__ CUtensorMap ropemap, const LatentArgs a) {
     using C = LatCfg<DC, TOK>;
@@ -65,6 +66,8 @@ __global__ void __launch_bounds__(256, 1)
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
     __shared__ uint32_t tmem_sh;
+    __shared__ uint64_t xbar;                 // row-value exchange between the two column halves
+    __shared__ float xchg_sh[2][2][128];
 
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *q_s = smem;
@@ -90,11 +93,12 @@ __global__ void __launch_bounds__(256, 1)
         mbar_init(&qempty_bar, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sfull_bar[s], 1);
-            mbar_init(&sfree_bar[s], 4);
-            mbar_init(&pfull_bar[s], 4);
+            mbar_init(&sfree_bar[s], 8);
+            mbar_init(&pfull_bar[s], 8);
             mbar_init(&pfree_bar[s], 1);
         }
         mbar_init(&end_bar, 1);
+        mbar_init(&xbar, 8);
         abort_sh = 0;
         fence_mbar_init();
     }
@@ -113,7 +117,7 @@ __global__ void __launch_bounds__(256, 1)
     // counters that persist across segment-list rounds
     uint32_t p_issued = 0, p_qloads = 0;                    // producer
     uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;        // MMA issuer
-    uint32_t x_tile = 0, x_s = 0, x_pv = 0;                 // softmax
+    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0;        // softmax
 
     for (int skip = 0;; skip += LMAXSEG) {
         if (warp == 0) {
@@ -199,7 +203,8 @@ __global__ void __launch_bounds__(256, 1)
             if (lane == 0) {
                 constexpr uint32_t idesc_s = umma_idesc_bf16(128, TOK, false, false);
                 constexpr uint32_t idesc_pv = umma_idesc_bf16(128, DV, false, true);
-                const uint32_t q_addr = smem_u32(q_s), st0 = smem_u32(stage_s);
+                const uint32_t st0 = smem_u32(stage_s);
+                const uint64_t dq0 = umma_desc(smem_u32(q_s), 16, 1024, 2);
                 bool ok = true;
                 auto issue_s = [&](uint32_t gt) -> bool {
                     const uint32_t stage = gt % nstage;
@@ -208,15 +213,14 @@ __global__ void __launch_bounds__(256, 1)
                     if (!mbar_wait_one(&sfree_bar[sb], ((m_s >> 1) & 1) ^ 1, &abort_sh, a.err, lim_ns)) return false;
                     tc_fence_after();
                     const uint32_t d = tmem + C::S_COL + sb * TOK;
-                    const uint32_t kv = st0 + stage * C::STAGE;
-#pragma unroll 1
+                    // descriptors advance by (byte offset >> 4) in their low word: one add per MMA
+                    const uint64_t dk0 = umma_desc(st0 + stage * C::STAGE, 16, 1024, 2);
+#pragma unroll
                     for (int kc = 0; kc < C::KCH; ++kc)
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t da = umma_desc(q_addr + kc * 16384 + kk * 32, 16, 1024, 2);
-                            const uint64_t db = umma_desc(kv + kc * C::CHUNK + kk * 32, 16, 1024, 2);
-                            umma_bf16(d, da, db, idesc_s, (kc | kk) != 0);
-                        }
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d, dq0 + (uint64_t)((kc * 16384 + kk * 32) >> 4),
+                                      dk0 + (uint64_t)((kc * C::CHUNK + kk * 32) >> 4), idesc_s, (kc | kk) != 0);
                     umma_commit(&sfull_bar[sb]);
                     ++m_s;
                     return true;
@@ -243,13 +247,12 @@ __global__ void __launch_bounds__(256, 1)
                         }
                         tc_fence_after();
                         const uint32_t stage = (m_tile + j) % nstage;
-                        const uint32_t v0 = st0 + stage * C::STAGE + vc * 4 * C::CHUNK;
+                        const uint64_t dv0 = umma_desc(st0 + stage * C::STAGE + vc * 4 * C::CHUNK, C::CHUNK, 1024, 2);
                         const uint32_t pa = tmem + C::P_COL + pb * C::P_COLS;
 #pragma unroll
-                        for (int kk = 0; kk < TOK / 16; ++kk) {
-                            const uint64_t db = umma_desc(v0 + kk * 2048, C::CHUNK, 1024, 2);
-                            umma_bf16_ts(tmem, pa + kk * 8, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                        }
+                        for (int kk = 0; kk < TOK / 16; ++kk)
+                            umma_bf16_ts(tmem, pa + kk * 8, dv0 + (uint64_t)(kk * 128), idesc_pv,
+                                         (j > 0 || kk > 0) ? 1u : 0u);
                         umma_commit(&pfree_bar[pb]);
                         umma_commit(&empty_bar[stage]);
                         ++m_pv;
@@ -260,10 +263,18 @@ __global__ void __launch_bounds__(256, 1)
             __syncwarp();
         } else if (warp >= 4) {
             // ================================================================ softmax / epilogue
-            const int r = threadIdx.x - 128;
+            // Eight warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 (its rows) and the column
+            // half hf = (w - 4) / 4 of every S tile, of P and of O.  The two threads of a row
+            // exchange their tile maxima through shared memory so that they keep the same
+            // reference maximum; their partial sums are merged in the epilogue.
+            constexpr int HC = TOK / 2;                  // S / P columns per thread
+            const int st_id = threadIdx.x - 128;         // 0..255
+            const int hf = (warp - 4) >> 2;
+            const int r = (warp & 3) * 32 + lane;        // row = TMEM lane
             const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
             const int n_row = rt * 128 + r;
             const bool row_ok = n_row < R;
+            const bool warp_live = rt * 128 + (warp & 3) * 32 < R;  // some row of this warp is real
             const int i_row = row_ok ? n_row / g : 0;
             const int head = row_ok ? c * g + n_row % g : 0;
             bool ok = true;
@@ -271,51 +282,67 @@ __global__ void __launch_bounds__(256, 1)
             auto wait_pv = [&](uint32_t k) -> bool {
                 return mbar_wait_warp(&pfree_bar[k & 1], (k >> 1) & 1, &abort_sh, a.err, lim_ns);
             };
+            // exchange one float per row with the other column half (bounded barrier over the 8 warps)
+            auto exchange = [&](float v, float &other) -> bool {
+                const int buf = x_x & 1;
+                xchg_sh[buf][hf][r] = v;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xbar);
+                if (!mbar_wait_warp(&xbar, x_x & 1, &abort_sh, a.err, lim_ns)) return false;
+                other = xchg_sh[buf][hf ^ 1][r];
+                ++x_x;
+                return true;
+            };
             for (int si = 0; si < nseg && ok; ++si) {
                 const Seg sg = segs[si];
                 const int b = sg.b;
                 const int T = clamp_len(__ldg(a.seqlens + b), max_tokens, a.L, nullptr);
                 const int lim = row_ok ? T - a.L + i_row : -1;
                 // l: sum of the fp32 P (gives lse); lq: sum of the bf16-rounded P the product
-                // uses (normalises O: a convex combination of the rounded weights).
+                // uses (normalises O: a convex combination of the rounded weights).  Both are
+                // partial over this thread's columns until the epilogue.
                 float m_ref = -INFINITY, l = 0.f, lq = 0.f;
                 for (int tile = sg.t0; tile < sg.t1; ++tile) {
-                    const int tok0 = tile * TOK;
+                    const int tok0 = tile * TOK + hf * HC;       // first token of this thread's columns
                     const uint32_t sb = x_s & 1;
                     if (!mbar_wait_warp(&sfull_bar[sb], (x_s >> 1) & 1, &abort_sh, a.err, lim_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    float s[TOK];
-                    {
-                        float tmp[32];
-                        tmem_ld32(tmem + lane_base + C::S_COL + sb * TOK, tmp);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) s[k] = tmp[k];
-                        if constexpr (TOK == 64) {
-                            tmem_ld32(tmem + lane_base + C::S_COL + sb * TOK + 32, tmp);
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) s[32 + k] = tmp[k];
+                    float s[HC];
+                    float mx = -INFINITY;
+                    if (warp_live) {
+                        if constexpr (HC == 32) {
+                            tmem_ld32(tmem + lane_base + C::S_COL + sb * TOK + hf * HC, s);
+                        } else {
+                            tmem_ld16(tmem + lane_base + C::S_COL + sb * TOK + hf * HC, s);
                         }
                     }
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sfree_bar[sb]);
                     ++x_s;
-
-                    float mx = -INFINITY;
+                    if (warp_live) {
+                        const bool full = tile * TOK + TOK - 1 <= T - a.L && row_ok;
 #pragma unroll
-                    for (int k = 0; k < TOK; ++k) {
-                        const float v = (tok0 + k <= lim) ? s[k] * a.scale_log2 : -INFINITY;
-                        s[k] = v;
-                        mx = fmaxf(mx, v);
+                        for (int k = 0; k < HC; ++k) {
+                            const float v = (full || tok0 + k <= lim) ? s[k] * a.scale_log2 : -INFINITY;
+                            s[k] = v;
+                            mx = fmaxf(mx, v);
+                        }
                     }
+                    float mo;
+                    if (!exchange(mx, mo)) {
+                        ok = false;
+                        break;
+                    }
+                    mx = fmaxf(mx, mo);
                     float alpha = 1.f;
                     bool need = false;
                     if (mx != -INFINITY) {
                         if (m_ref == -INFINITY) {
-                            m_ref = mx;  // nothing visible before: O and l hold zeros
+                            m_ref = mx;  // nothing visible before: O and the sums hold zeros
                         } else if (mx > m_ref + RESCALE_LOG2) {
                             alpha = ex2(m_ref - mx);
                             need = true;
@@ -332,63 +359,67 @@ __global__ void __launch_bounds__(256, 1)
                         l *= alpha;
                         lq *= alpha;
 #pragma unroll 1
-                        for (int ch = 0; ch < DV / 32; ++ch) {
+                        for (int ch = 0; ch < DV / 64; ++ch) {
                             float o[32];
-                            tmem_ld32(tmem + lane_base + ch * 32, o);
+                            const uint32_t col = hf * (DV / 2) + ch * 32;
+                            tmem_ld32(tmem + lane_base + col, o);
 #pragma unroll
                             for (int k = 0; k < 32; ++k) o[k] *= alpha;
-                            tmem_st32(tmem + lane_base + ch * 32, o);
+                            tmem_st32(tmem + lane_base + col, o);
                         }
                         tmem_st_wait();
                     }
-                    if (m_ref != -INFINITY) {
+                    if (warp_live) {
+                        if (m_ref != -INFINITY) {
 #pragma unroll
-                        for (int k = 0; k < TOK; ++k) {
-                            s[k] = ex2(s[k] - m_ref);
-                            l += s[k];
+                            for (int k = 0; k < HC; ++k) {
+                                s[k] = ex2(s[k] - m_ref);
+                                l += s[k];
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < HC; ++k) s[k] = 0.f;
                         }
-                    } else {
-#pragma unroll
-                        for (int k = 0; k < TOK; ++k) s[k] = 0.f;
                     }
 
                     // tokens past T_b in this tile hold garbage: zero their value rows (P is 0 there,
                     // but 0 * NaN would still poison the product)
                     const uint32_t stage = x_tile % nstage;
-                    if (tok0 + TOK > T) {
-                        const int k0 = max(T - tok0, 0);
+                    const int ttok0 = tile * TOK;
+                    if (ttok0 + TOK > T) {
+                        const int k0 = max(T - ttok0, 0);
                         uint8_t *v0 = stage_s + (size_t)stage * C::STAGE + (size_t)vc * 4 * C::CHUNK;
                         const int units = (TOK - k0) * 4 * 8;  // 16-byte units: rows x 4 chunks x 8
-                        for (int u = r; u < units; u += 128) {
+                        for (int u = st_id; u < units; u += 256) {
                             const int row = k0 + u / 32, ch = (u / 8) & 3, k = u & 7;
                             *(uint4 *)(v0 + ch * C::CHUNK + row * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                         }
                     }
-                    // P row (bf16 pairs) -> tensor memory buffer x_pv & 1, once the P.V that last
-                    // read that buffer has completed.  The normaliser sums the same rounded values
-                    // the product uses.
+                    // P (bf16 pairs) -> tensor memory buffer x_pv & 1, once the P.V that last read
+                    // that buffer has completed
                     if (x_pv >= 2 && !wait_pv(x_pv - 2)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    float sum = 0.f;
-                    {
-                        const uint32_t pa = tmem + lane_base + C::P_COL + (x_pv & 1) * C::P_COLS;
+                    if (warp_live) {
+                        const uint32_t pa = tmem + lane_base + C::P_COL + (x_pv & 1) * C::P_COLS + hf * (HC / 2);
+                        uint32_t w[HC / 2];
+                        float sum = 0.f;
 #pragma unroll
-                        for (int h = 0; h < TOK / 32; ++h) {
-                            uint32_t w[16];
-#pragma unroll
-                            for (int k = 0; k < 16; ++k) {
-                                w[k] = pack_bf16(s[32 * h + 2 * k], s[32 * h + 2 * k + 1]);
-                                sum += bf16_lo(w[k]) + bf16_hi(w[k]);
-                            }
-                            tmem_st16u(pa + 16 * h, w);
+                        for (int k = 0; k < HC / 2; ++k) {
+                            w[k] = pack_bf16(s[2 * k], s[2 * k + 1]);
+                            sum += bf16_lo(w[k]) + bf16_hi(w[k]);
+                        }
+                        if constexpr (HC == 32) {
+                            tmem_st16u(pa, w);
+                        } else {
+                            tmem_st8u(pa, w);
                         }
                         tmem_st_wait();
+                        lq += sum;
                     }
-                    lq += sum;
-                    if (tok0 + TOK > T) fence_proxy_async();  // the zeroed value rows above
+                    if (ttok0 + TOK > T) fence_proxy_async();  // the zeroed value rows above
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&pfull_bar[x_pv & 1]);
@@ -397,7 +428,14 @@ __global__ void __launch_bounds__(256, 1)
                 }
                 if (!ok) break;
 
-                // ---- epilogue: O is final once the last P.V completes
+                // ---- epilogue: merge the two halves' sums; O is final once the last P.V completes
+                float lo, lqo;
+                if (!exchange(l, lo) || !exchange(lq, lqo)) {
+                    ok = false;
+                    break;
+                }
+                l += lo;
+                lq += lqo;
                 if (!wait_pv(x_pv - 1)) {
                     ok = false;
                     break;
@@ -407,28 +445,32 @@ __global__ void __launch_bounds__(256, 1)
                 const float lse_v = l > 0.f ? (m_ref + lg2(l)) * 0.69314718055994530942f : -INFINITY;
                 const size_t rows_b = (size_t)a.L * a.h_q;
                 const size_t r_out = (size_t)i_row * a.h_q + head;
+                if (warp_live) {
 #pragma unroll 1
-                for (int ch = 0; ch < DV / 32; ++ch) {
-                    float o[32];
-                    tmem_ld32(tmem + lane_base + ch * 32, o);
-                    if (!row_ok) continue;
-                    if (sg.nsplit == 1) {
-                        uint4 *op = (uint4 *)(a.out + ((size_t)b * rows_b + r_out) * DC + vc * DV + ch * 32);
+                    for (int ch = 0; ch < DV / 64; ++ch) {
+                        float o[32];
+                        const int col = hf * (DV / 2) + ch * 32;
+                        tmem_ld32(tmem + lane_base + col, o);
+                        if (!row_ok) continue;
+                        if (sg.nsplit == 1) {
+                            uint4 *op = (uint4 *)(a.out + ((size_t)b * rows_b + r_out) * DC + vc * DV + col);
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            op[k] = make_uint4(pack_bf16(o[8 * k] * inv, o[8 * k + 1] * inv),
-                                               pack_bf16(o[8 * k + 2] * inv, o[8 * k + 3] * inv),
-                                               pack_bf16(o[8 * k + 4] * inv, o[8 * k + 5] * inv),
-                                               pack_bf16(o[8 * k + 6] * inv, o[8 * k + 7] * inv));
-                    } else {
-                        float4 *op = (float4 *)(a.ws_o + ((size_t)sg.slot * rows_b + r_out) * DC + vc * DV + ch * 32);
+                            for (int k = 0; k < 4; ++k)
+                                op[k] = make_uint4(pack_bf16(o[8 * k] * inv, o[8 * k + 1] * inv),
+                                                   pack_bf16(o[8 * k + 2] * inv, o[8 * k + 3] * inv),
+                                                   pack_bf16(o[8 * k + 4] * inv, o[8 * k + 5] * inv),
+                                                   pack_bf16(o[8 * k + 6] * inv, o[8 * k + 7] * inv));
+                        } else {
+                            float4 *op =
+                                (float4 *)(a.ws_o + ((size_t)sg.slot * rows_b + r_out) * DC + vc * DV + col);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            op[k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv,
-                                                o[4 * k + 3] * inv);
+                            for (int k = 0; k < 8; ++k)
+                                op[k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv,
+                                                    o[4 * k + 3] * inv);
+                        }
                     }
                 }
-                if (row_ok && vc == 0) {
+                if (row_ok && vc == 0 && hf == 0) {
                     if (sg.nsplit == 1)
                         a.lse[(size_t)b * rows_b + r_out] = lse_v;
                     else
@@ -460,7 +502,7 @@ cudaError_t launch_t(const CUtensorMap &qm, const CUtensorMap &lm, const CUtenso
     auto k = latent_decode_kernel<DC, TOK>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, 256, smem, st>>>(qm, lm, rm, a);
+    k<<<grid, 384, smem, st>>>(qm, lm, rm, a);
     return cudaGetLastError();
 }
 
