@@ -226,6 +226,7 @@ constexpr size_t LATENT_STATIC_SMEM = 4096;
 
 struct LatentPlan {
     LatentShape shape;
+    bool pair;
     int n_rt, n_vc, n_sub, parts, nstage, rb;
     size_t smem, ws_bytes;
 };
@@ -252,8 +253,10 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
         return KVD_ERR_UNSUPPORTED_SHAPE;
     lp->shape = sh;
     lp->n_rt = (int)((R + 127) / 128);
-    lp->n_vc = p->d_c / 256;
+    lp->pair = p->d_c == 512;  // CTA pairs split the key dimension instead of the value
+    lp->n_vc = lp->pair ? 1 : p->d_c / 256;
     lp->n_sub = p->h_c * lp->n_rt * lp->n_vc;
+    const int ctas_per_sub = lp->pair ? 2 : 1;
     lp->rb = g < 128 ? g : 128;
     const size_t fixed = SMEM_PER_BLOCK - LATENT_STATIC_SMEM - 1024 - sh.q_bytes - sh.p_bytes;
     int nstage = (int)(fixed / sh.stage_bytes);
@@ -265,7 +268,7 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
     if (parts == 0) {
         const int sms = num_sms_current();
         if (sms <= 0) return KVD_ERR_CUDA;
-        parts = sms / lp->n_sub > 0 ? sms / lp->n_sub : 1;
+        parts = sms / (lp->n_sub * ctas_per_sub) > 0 ? sms / (lp->n_sub * ctas_per_sub) : 1;
     }
     lp->parts = parts;
     const size_t slots = (size_t)p->B + parts - 1;
@@ -331,8 +334,32 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     a.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
     a.debug_flags = g_debug_flags.load();
     record(g_ev_before, st);
-    if (launch_latent_decode(p->d_c, qm, lm, rm, a, lp.parts * lp.n_sub, lp.smem, st) != cudaSuccess)
+    if (lp.pair) {
+        CUtensorMap qrm, lm2, rm2;
+        {   // q's rope dims in 32-wide halves (64-byte rows, 64 B swizzle)
+            cuuint64_t dims[3] = {32, (cuuint64_t)p->B * p->L * p->h_q, (cuuint64_t)d_qk / 32};
+            cuuint64_t strides[2] = {(cuuint64_t)d_qk * 2, 64};
+            cuuint32_t box[3] = {32, (cuuint32_t)lp.rb, 1};
+            if (!encode(&qrm, p->q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B)) return KVD_ERR_CUDA;
+        }
+        {   // four 64-wide latent chunks (one CTA's half of a latent head) per box
+            cuuint64_t dims[3] = {64, tokens, (cuuint64_t)p->h_c * p->d_c / 64};
+            cuuint64_t strides[2] = {(cuuint64_t)p->h_c * p->d_c * 2, 128};
+            cuuint32_t box[3] = {64, (cuuint32_t)lp.shape.tok, 4};
+            if (!encode(&lm2, p->latent_cache, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                return KVD_ERR_CUDA;
+        }
+        {   // 32-wide halves of the rope rows
+            cuuint64_t dims[2] = {64, tokens};
+            cuuint64_t strides[1] = {128};
+            cuuint32_t box[2] = {32, (cuuint32_t)lp.shape.tok};
+            if (!encode(&rm2, p->rope_cache, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B)) return KVD_ERR_CUDA;
+        }
+        if (launch_mla_pair(qm, qrm, lm2, rm2, a, lp.parts * lp.n_sub * 2, lp.smem, st) != cudaSuccess)
+            return KVD_ERR_CUDA;
+    } else if (launch_latent_decode(p->d_c, qm, lm, rm, a, lp.parts * lp.n_sub, lp.smem, st) != cudaSuccess) {
         return KVD_ERR_CUDA;
+    }
     record(g_ev_after, st);
 
     CombineArgs c;

@@ -415,3 +415,77 @@ __device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&v)[8]
 }
 }  // namespace kvd
 #endif  // __CUDACC__
+
+#ifdef __CUDACC__
+namespace kvd {
+// ----------------------------------------------------------------------------- thread-block clusters
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// The shared::cluster address of `saddr` (a shared::cta address) in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster, releasing this thread's prior writes.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr_bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// As mbar_wait_warp, acquiring at cluster scope (for barriers that another CTA arrives on).
+__device__ __forceinline__ bool mbar_wait_warp_cluster(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                       uint32_t *err, uint64_t limit_ns) {
+    if (__all_sync(0xffffffffu, mbar_try_wait_cluster(bar, parity))) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (__all_sync(0xffffffffu, mbar_try_wait_cluster(bar, parity))) return true;
+        int stop = 0;
+        if ((threadIdx.x & 31) == 0) {
+            if (*abort) {
+                stop = 1;
+            } else if (globaltimer() - t0 > limit_ns) {
+                set_error(err, DEVERR_TIMEOUT);
+                *abort = 1;
+                stop = 1;
+            }
+        }
+        if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+    }
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+}  // namespace kvd
+#endif  // __CUDACC__
+
+#ifdef __CUDACC__
+namespace kvd {
+// Asynchronous store of 16 bytes into another CTA's shared memory; completes `bytes` of the
+// transaction count of that CTA's mbarrier at caddr_bar (same CTA as the destination).
+__device__ __forceinline__ void st_async_v4(uint32_t caddr, float a, float b, float c, float d, uint32_t caddr_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                     caddr),
+                 "f"(a), "f"(b), "f"(c), "f"(d), "r"(caddr_bar)
+                 : "memory");
+}
+}  // namespace kvd
+#endif  // __CUDACC__

@@ -70,6 +70,12 @@ LatentShape latent_shape(int d_c);
 cudaError_t launch_latent_decode(int d_c, const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
                                  const LatentArgs &a, int grid, size_t smem, cudaStream_t st);
 
+// d_c = 512 (MLA): CTA pairs splitting the key dimension (latent_pair.cu).
+uint32_t mla_pair_fixed_smem();   // q half + the exchange buffer
+uint32_t mla_pair_stage_bytes();  // one 64-token tile half
+cudaError_t launch_mla_pair(const CUtensorMap &qm, const CUtensorMap &qrm, const CUtensorMap &lm,
+                            const CUtensorMap &rm, const LatentArgs &a, int grid, size_t smem, cudaStream_t st);
+
 struct CombineArgs {
     const int32_t *seqlens;
     const float *ws_lse;

@@ -515,10 +515,10 @@ LatentShape latent_shape(int d_c) {
         s.q_bytes = LatCfg<256, 64>::Q_BYTES;
         s.stage_bytes = LatCfg<256, 64>::STAGE;
         s.p_bytes = 0;
-    } else if (d_c == 512) {
-        s.tok = 32;
-        s.q_bytes = LatCfg<512, 32>::Q_BYTES;
-        s.stage_bytes = LatCfg<512, 32>::STAGE;
+    } else if (d_c == 512) {  // the CTA-pair kernel of latent_pair.cu
+        s.tok = 64;
+        s.q_bytes = mla_pair_fixed_smem();
+        s.stage_bytes = mla_pair_stage_bytes();
         s.p_bytes = 0;
     }
     return s;
@@ -527,7 +527,6 @@ LatentShape latent_shape(int d_c) {
 cudaError_t launch_latent_decode(int d_c, const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
                                  const LatentArgs &a, int grid, size_t smem, cudaStream_t st) {
     if (d_c == 256) return launch_t<256, 64>(qm, lm, rm, a, grid, smem, st);
-    if (d_c == 512) return launch_t<512, 32>(qm, lm, rm, a, grid, smem, st);
     return cudaErrorInvalidValue;
 }
 

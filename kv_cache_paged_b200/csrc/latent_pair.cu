@@ -1,0 +1,522 @@
+// MLA decode (absorbed, d_c = 512) on a pair of CTAs that split the key dimension.
+//
+// "Hardware-Efficient Attention for Fast Decoding", section 3.3.2 with h_c latent heads of
+// width d_c = 512 (MLA: h_c = 1).  The fp32 accumulator of 128 query rows x 512 value
+// columns alone fills tensor memory, so the value columns are split over two CTAs.  Rather
+// than have both CTAs compute the same 128 x 576 score product, the pair (a thread-block
+// cluster of 2) splits the 576-wide key dimension as well: CTA k holds q's latent dims
+// [256k, 256k + 256) and rope dims [32k, 32k + 32) (72 KB of shared memory instead of 144 KB),
+// loads only those columns of each 64-token tile (36 KB), computes a partial score
+// S_k = Q_k K_k^T on tcgen05 and swaps it with its peer through distributed shared memory.
+// Both CTAs then hold the same S = S_0 + S_1 (fp32 addition commutes, so the sums agree bit
+// for bit), run the same softmax and accumulate O for their own 256 latent columns, which are
+// exactly the latent columns they loaded.  Every byte of the cache is read once per pair.
+//
+// Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4..11 softmax
+// (two threads per row, one per 32-token half of the tile).  Tensor memory: O [0, 256),
+// two partial-S buffers [256, 384), two P buffers [384, 448).  Every wait is bounded.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvd {
+
+namespace {
+
+constexpr int PMAXSEG = 32;
+constexpr int PTOK = 64;                                  // tokens per tile
+constexpr int PDV = 256;                                  // value columns per CTA
+constexpr uint32_t P_QLAT = 4 * 16384;                    // q latent half: 4 chunks x 128 rows x 128 B
+constexpr uint32_t P_QBYTES = P_QLAT + 128 * 64;          // + rope half: 128 rows x 64 B
+constexpr uint32_t P_CHUNK = PTOK * 128;                  // one 64-dim chunk of a tile
+constexpr uint32_t P_STAGE = 4 * P_CHUNK + PTOK * 64;     // latent half + rope half
+constexpr uint32_t P_XBYTES = 128 * 64 * 4;               // the peer's partial S (fp32)
+constexpr uint32_t P_SCOL = PDV, P_PCOL = PDV + 2 * PTOK, P_PCOLS = PTOK / 2;
+constexpr float P_RESCALE_LOG2 = 8.f;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
+    mla_pair_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap qrmap,
+                    const __grid_constant__ CUtensorMap latmap, const __grid_constant__ CUtensorMap ropemap,
+                    const LatentArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
+    __shared__ uint64_t qfull_bar, qempty_bar, sfull_bar[2], sfree_bar[2], pfull_bar[2], pfree_bar[2], end_bar;
+    __shared__ uint64_t xbar, xfull_bar, xfree_bar;
+    __shared__ Seg segs[PMAXSEG];
+    __shared__ int nseg_sh, more_sh;
+    __shared__ volatile int abort_sh;
+    __shared__ uint32_t tmem_sh;
+    __shared__ float xchg_sh[2][2][128];
+
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *q_s = smem;
+    uint8_t *xbuf_s = smem + P_QBYTES;                      // receives the peer's partial S
+    uint8_t *stage_s = xbuf_s + P_XBYTES;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t kr = cluster_rank();                     // 0 or 1: which half of the key
+    const uint32_t peer = kr ^ 1u;
+    const int pair = blockIdx.x >> 1;
+    const int part = pair / a.n_sub, sub = pair % a.n_sub;
+    const int rt = sub % a.n_rt;
+    const int c = sub / a.n_rt;
+    const int g = a.h_q / a.h_c;
+    const int R = g * a.L;
+    const int max_tokens = a.max_pages * a.page_size;
+    const int nstage = a.nstage;
+    const uint64_t lim_ns = a.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nstage; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&qfull_bar, 1);
+        mbar_init(&qempty_bar, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sfull_bar[s], 1);
+            mbar_init(&sfree_bar[s], 8);
+            mbar_init(&pfull_bar[s], 8);
+            mbar_init(&pfree_bar[s], 1);
+        }
+        mbar_init(&end_bar, 1);
+        mbar_init(&xbar, 8);
+        // xfull: one local arrival that arms the expected bytes, completed by the peer's st.async
+        // (32 KB per tile); xfree: one arrival from each of the peer's 8 softmax warps
+        mbar_init(&xfull_bar, 1);
+        mbar_init(&xfree_bar, 8);
+        mbar_arrive_expect_tx(&xfull_bar, P_XBYTES);  // arm the first tile's exchange
+        abort_sh = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&tmem_sh, 512);
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&qmap);
+        tma_prefetch_desc(&qrmap);
+        tma_prefetch_desc(&latmap);
+        tma_prefetch_desc(&ropemap);
+    }
+    pdl_launch_dependents();
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers are initialised before any remote arrival
+    tc_fence_after();
+    const uint32_t tmem = tmem_sh;
+
+    uint32_t p_issued = 0, p_qloads = 0;
+    uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;
+    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0, x_p = 0;
+
+    for (int skip = 0;; skip += PMAXSEG) {
+        if (warp == 0) {
+            int cnt = 0;
+            plan_walk(a.seqlens, a.B, PTOK, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
+                if (cnt >= skip && cnt < skip + PMAXSEG) segs[cnt - skip] = s;
+                ++cnt;
+            });
+            if (lane == 0) {
+                nseg_sh = cnt - skip < PMAXSEG ? (cnt - skip > 0 ? cnt - skip : 0) : PMAXSEG;
+                more_sh = cnt > skip + PMAXSEG;
+            }
+        }
+        __syncthreads();
+        const int nseg = nseg_sh;
+
+        if (warp == 0) {
+            // ================================================================ producer
+            const uint64_t pol = policy_evict_first();
+            bool stop = false;
+            const int rb = g < 128 ? g : 128;
+            const int rows_tile = min(R - rt * 128, 128);
+            for (int si = 0; si < nseg && !stop; ++si) {
+                const Seg sg = segs[si];
+                if (!mbar_wait_warp(&qempty_bar, (p_qloads & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&qfull_bar, (uint32_t)rows_tile * (4 * 128 + 64));
+                    for (int run = 0; run * rb < rows_tile; ++run) {
+                        const int n0 = rt * 128 + run * rb;
+                        const int i = n0 / g, h0 = n0 % g;
+                        const int row = (sg.b * a.L + i) * a.h_q + c * g + h0;
+                        for (int ch = 0; ch < 4; ++ch)
+                            tma_load_3d(q_s + ch * 16384 + run * rb * 128, &qmap, &qfull_bar, 0, row, 4 * kr + ch,
+                                        pol);
+                        tma_load_3d(q_s + P_QLAT + run * rb * 64, &qrmap, &qfull_bar, 0, row, 16 + kr, pol);
+                    }
+                }
+                ++p_qloads;
+                const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
+                const int tpp = a.page_size / PTOK;
+                const int p_first = sg.t0 / tpp, p_last = (sg.t1 - 1) / tpp;
+                for (int pb = p_first; pb <= p_last && !stop; pb += 32) {
+                    int page = 0;
+                    if (pb + lane <= p_last) {
+                        page = __ldg(bt + pb + lane);
+                        if (page < 0 || page >= a.num_pages) {
+                            set_error(a.err, DEVERR_BAD_PAGE);
+                            page = 0;
+                        }
+                    }
+                    const int t_lo = max(sg.t0, pb * tpp), t_hi = min(sg.t1, (pb + 32) * tpp);
+                    for (int t = t_lo; t < t_hi; ++t) {
+                        const int pg = __shfl_sync(0xffffffffu, page, t / tpp - pb);
+                        const uint32_t stage = p_issued % nstage;
+                        if (!mbar_wait_warp(&empty_bar[stage], ((p_issued / nstage) & 1) ^ 1, &abort_sh, a.err,
+                                            lim_ns)) {
+                            stop = true;
+                            break;
+                        }
+                        if (lane == 0) {
+                            uint8_t *st = stage_s + (size_t)stage * P_STAGE;
+                            const int row = pg * a.page_size + (t % tpp) * PTOK;
+                            mbar_arrive_expect_tx(&full_bar[stage], P_STAGE);
+                            if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0) {
+                                tma_load_3d(st, &latmap, &full_bar[stage], 0, row, c * 8 + 4 * kr, pol);
+                                tma_load_2d(st + 4 * P_CHUNK, &ropemap, &full_bar[stage], 32 * kr, row, pol);
+                            }
+                        }
+                        ++p_issued;
+                    }
+                }
+            }
+            if (stop) {
+                volatile int never = 0;
+                const uint32_t lo = p_issued > (uint32_t)nstage ? p_issued - nstage : 0;
+                for (uint32_t k = lo; k < p_issued; ++k)
+                    mbar_wait_warp(&full_bar[k % nstage], (k / nstage) & 1, &never, nullptr, lim_ns);
+                if (p_qloads) mbar_wait_warp(&qfull_bar, (p_qloads - 1) & 1, &never, nullptr, lim_ns);
+            }
+        } else if (warp == 1) {
+            // ================================================================ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idesc_s = umma_idesc_bf16(128, PTOK, false, false);
+                constexpr uint32_t idesc_pv = umma_idesc_bf16(128, PDV, false, true);
+                const uint32_t st0 = smem_u32(stage_s);
+                const uint64_t dq0 = umma_desc(smem_u32(q_s), 16, 1024, 2);          // latent, 128 B swizzle
+                const uint64_t dqr = umma_desc(smem_u32(q_s) + P_QLAT, 16, 512, 4);  // rope half, 64 B swizzle
+                bool ok = true;
+                auto issue_s = [&](uint32_t gt) -> bool {
+                    const uint32_t stage = gt % nstage;
+                    if (!mbar_wait_one(&full_bar[stage], (gt / nstage) & 1, &abort_sh, a.err, lim_ns)) return false;
+                    const uint32_t sb = m_s & 1;
+                    if (!mbar_wait_one(&sfree_bar[sb], ((m_s >> 1) & 1) ^ 1, &abort_sh, a.err, lim_ns)) return false;
+                    tc_fence_after();
+                    const uint32_t d = tmem + P_SCOL + sb * PTOK;
+                    const uint64_t dk0 = umma_desc(st0 + stage * P_STAGE, 16, 1024, 2);
+                    const uint64_t dkr = umma_desc(st0 + stage * P_STAGE + 4 * P_CHUNK, 16, 512, 4);
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d, dq0 + (uint64_t)((ch * 16384 + kk * 32) >> 4),
+                                      dk0 + (uint64_t)((ch * P_CHUNK + kk * 32) >> 4), idesc_s, (ch | kk) != 0);
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk)
+                        umma_bf16(d, dqr + (uint64_t)(kk * 2), dkr + (uint64_t)(kk * 2), idesc_s, 1u);
+                    umma_commit(&sfull_bar[sb]);
+                    ++m_s;
+                    return true;
+                };
+                for (int si = 0; si < nseg && ok; ++si) {
+                    const int n = segs[si].t1 - segs[si].t0;
+                    if (!mbar_wait_one(&qfull_bar, m_q & 1, &abort_sh, a.err, lim_ns)) break;
+                    ++m_q;
+                    tc_fence_after();
+                    if (!issue_s(m_tile)) break;
+                    if (n == 1) umma_commit(&qempty_bar);
+                    for (int j = 0; j < n; ++j) {
+                        if (j + 1 < n) {
+                            if (!issue_s(m_tile + j + 1)) {
+                                ok = false;
+                                break;
+                            }
+                            if (j + 1 == n - 1) umma_commit(&qempty_bar);
+                        }
+                        const uint32_t pb = m_pv & 1;
+                        if (!mbar_wait_one(&pfull_bar[pb], (m_pv >> 1) & 1, &abort_sh, a.err, lim_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t stage = (m_tile + j) % nstage;
+                        const uint64_t dv0 = umma_desc(st0 + stage * P_STAGE, P_CHUNK, 1024, 2);
+                        const uint32_t pa = tmem + P_PCOL + pb * P_PCOLS;
+#pragma unroll
+                        for (int kk = 0; kk < PTOK / 16; ++kk)
+                            umma_bf16_ts(tmem, pa + kk * 8, dv0 + (uint64_t)(kk * 128), idesc_pv,
+                                         (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&pfree_bar[pb]);
+                        umma_commit(&empty_bar[stage]);
+                        ++m_pv;
+                    }
+                    m_tile += n;
+                }
+            }
+            __syncwarp();
+        } else if (warp >= 4) {
+            // ================================================================ softmax / epilogue
+            constexpr int HC = PTOK / 2;
+            const int st_id = threadIdx.x - 128;
+            const int hf = (warp - 4) >> 2;
+            const int r = (warp & 3) * 32 + lane;
+            const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+            const int n_row = rt * 128 + r;
+            const bool row_ok = n_row < R;
+            const bool warp_live = rt * 128 + (warp & 3) * 32 < R;
+            const int i_row = row_ok ? n_row / g : 0;
+            const int head = row_ok ? c * g + n_row % g : 0;
+            // my row of the exchange buffer, as this CTA and as the peer addresses it
+            const uint32_t x_row = smem_u32(xbuf_s) + r * 256;
+            const uint32_t x_row_peer = mapa_shared(x_row, peer);
+            const uint32_t peer_xfull = mapa_shared(smem_u32(&xfull_bar), peer);
+            const uint32_t peer_xfree = mapa_shared(smem_u32(&xfree_bar), peer);
+            bool ok = true;
+            auto wait_pv = [&](uint32_t k) -> bool {
+                return mbar_wait_warp(&pfree_bar[k & 1], (k >> 1) & 1, &abort_sh, a.err, lim_ns);
+            };
+            auto exchange = [&](float v, float &other) -> bool {
+                const int buf = x_x & 1;
+                xchg_sh[buf][hf][r] = v;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xbar);
+                if (!mbar_wait_warp(&xbar, x_x & 1, &abort_sh, a.err, lim_ns)) return false;
+                other = xchg_sh[buf][hf ^ 1][r];
+                ++x_x;
+                return true;
+            };
+            for (int si = 0; si < nseg && ok; ++si) {
+                const Seg sg = segs[si];
+                const int b = sg.b;
+                const int T = clamp_len(__ldg(a.seqlens + b), max_tokens, a.L, nullptr);
+                const int lim = row_ok ? T - a.L + i_row : -1;
+                float m_ref = -INFINITY, l = 0.f, lq = 0.f;
+                for (int tile = sg.t0; tile < sg.t1; ++tile) {
+                    const int tok0 = tile * PTOK + hf * HC;
+                    const uint32_t sb = x_s & 1;
+                    if (!mbar_wait_warp(&sfull_bar[sb], (x_s >> 1) & 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    float s[HC];
+                    tmem_ld32(tmem + lane_base + P_SCOL + sb * PTOK + hf * HC, s);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sfree_bar[sb]);
+                    ++x_s;
+
+                    // ---- swap partial scores with the peer CTA (fp32, distributed shared memory)
+                    if (x_p > 0 && !mbar_wait_warp_cluster(&xfree_bar, (x_p - 1) & 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int c4 = 0; c4 < HC / 4; ++c4) {
+                        const uint32_t c16 = hf * (HC / 4) + c4;
+                        st_async_v4(x_row_peer + ((c16 ^ (r & 15)) << 4), s[4 * c4], s[4 * c4 + 1], s[4 * c4 + 2],
+                                    s[4 * c4 + 3], peer_xfull);
+                    }
+                    if (!mbar_wait_warp_cluster(&xfull_bar, x_p & 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int c4 = 0; c4 < HC / 4; ++c4) {
+                        const uint32_t c16 = hf * (HC / 4) + c4;
+                        float4 v;
+                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                                     : "r"(x_row + ((c16 ^ (r & 15)) << 4))
+                                     : "memory");
+                        s[4 * c4] += v.x;
+                        s[4 * c4 + 1] += v.y;
+                        s[4 * c4 + 2] += v.z;
+                        s[4 * c4 + 3] += v.w;
+                    }
+                    // this warp's rows are read (the sums above used them): arm the next exchange,
+                    // then let the peer overwrite the buffer
+                    __syncwarp();
+                    if (threadIdx.x == 128) mbar_arrive_expect_tx(&xfull_bar, P_XBYTES);
+                    if (lane == 0) mbar_arrive_cluster(peer_xfree);
+                    ++x_p;
+
+                    float mx = -INFINITY;
+                    if (warp_live) {
+                        const bool full = tile * PTOK + PTOK - 1 <= T - a.L && row_ok;
+#pragma unroll
+                        for (int k = 0; k < HC; ++k) {
+                            const float v = (full || tok0 + k <= lim) ? s[k] * a.scale_log2 : -INFINITY;
+                            s[k] = v;
+                            mx = fmaxf(mx, v);
+                        }
+                    }
+                    float mo;
+                    if (!exchange(mx, mo)) {
+                        ok = false;
+                        break;
+                    }
+                    mx = fmaxf(mx, mo);
+                    float alpha = 1.f;
+                    bool need = false;
+                    if (mx != -INFINITY) {
+                        if (m_ref == -INFINITY) {
+                            m_ref = mx;
+                        } else if (mx > m_ref + P_RESCALE_LOG2) {
+                            alpha = ex2(m_ref - mx);
+                            need = true;
+                            m_ref = mx;
+                        }
+                    }
+                    if (__any_sync(0xffffffffu, need)) {
+                        if (x_pv > 0 && !wait_pv(x_pv - 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        l *= alpha;
+                        lq *= alpha;
+#pragma unroll 1
+                        for (int ch = 0; ch < PDV / 64; ++ch) {
+                            float o[32];
+                            const uint32_t col = hf * (PDV / 2) + ch * 32;
+                            tmem_ld32(tmem + lane_base + col, o);
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) o[k] *= alpha;
+                            tmem_st32(tmem + lane_base + col, o);
+                        }
+                        tmem_st_wait();
+                    }
+                    if (warp_live) {
+                        if (m_ref != -INFINITY) {
+#pragma unroll
+                            for (int k = 0; k < HC; ++k) {
+                                s[k] = ex2(s[k] - m_ref);
+                                l += s[k];
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < HC; ++k) s[k] = 0.f;
+                        }
+                    }
+                    // value rows of tokens past T_b hold garbage: zero them (0 * NaN would poison O)
+                    const uint32_t stage = x_tile % nstage;
+                    const int ttok0 = tile * PTOK;
+                    if (ttok0 + PTOK > T) {
+                        const int k0 = max(T - ttok0, 0);
+                        uint8_t *v0 = stage_s + (size_t)stage * P_STAGE;
+                        const int units = (PTOK - k0) * 4 * 8;
+                        for (int u = st_id; u < units; u += 256) {
+                            const int row = k0 + u / 32, ch = (u / 8) & 3, k = u & 7;
+                            *(uint4 *)(v0 + ch * P_CHUNK + row * 128 + k * 16) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    if (x_pv >= 2 && !wait_pv(x_pv - 2)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (warp_live) {
+                        const uint32_t pa = tmem + lane_base + P_PCOL + (x_pv & 1) * P_PCOLS + hf * (HC / 2);
+                        uint32_t w[HC / 2];
+                        float sum = 0.f;
+#pragma unroll
+                        for (int k = 0; k < HC / 2; ++k) {
+                            w[k] = pack_bf16(s[2 * k], s[2 * k + 1]);
+                            sum += bf16_lo(w[k]) + bf16_hi(w[k]);
+                        }
+                        tmem_st16u(pa, w);
+                        tmem_st_wait();
+                        lq += sum;
+                    }
+                    if (ttok0 + PTOK > T) fence_proxy_async();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pfull_bar[x_pv & 1]);
+                    ++x_pv;
+                    ++x_tile;
+                }
+                if (!ok) break;
+
+                float lo, lqo;
+                if (!exchange(l, lo) || !exchange(lq, lqo)) {
+                    ok = false;
+                    break;
+                }
+                l += lo;
+                lq += lqo;
+                if (!wait_pv(x_pv - 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float inv = lq > 0.f ? 1.f / lq : 0.f;
+                const float lse_v = l > 0.f ? (m_ref + lg2(l)) * 0.69314718055994530942f : -INFINITY;
+                const size_t rows_b = (size_t)a.L * a.h_q;
+                const size_t r_out = (size_t)i_row * a.h_q + head;
+                if (warp_live) {
+#pragma unroll 1
+                    for (int ch = 0; ch < PDV / 64; ++ch) {
+                        float o[32];
+                        const int col = hf * (PDV / 2) + ch * 32;
+                        tmem_ld32(tmem + lane_base + col, o);
+                        if (!row_ok) continue;
+                        const int gcol = kr * PDV + col;
+                        if (sg.nsplit == 1) {
+                            uint4 *op = (uint4 *)(a.out + ((size_t)b * rows_b + r_out) * 512 + gcol);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                op[k] = make_uint4(pack_bf16(o[8 * k] * inv, o[8 * k + 1] * inv),
+                                                   pack_bf16(o[8 * k + 2] * inv, o[8 * k + 3] * inv),
+                                                   pack_bf16(o[8 * k + 4] * inv, o[8 * k + 5] * inv),
+                                                   pack_bf16(o[8 * k + 6] * inv, o[8 * k + 7] * inv));
+                        } else {
+                            float4 *op = (float4 *)(a.ws_o + ((size_t)sg.slot * rows_b + r_out) * 512 + gcol);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                op[k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv,
+                                                    o[4 * k + 3] * inv);
+                        }
+                    }
+                }
+                if (row_ok && kr == 0 && hf == 0) {
+                    if (sg.nsplit == 1)
+                        a.lse[(size_t)b * rows_b + r_out] = lse_v;
+                    else
+                        a.ws_lse[(size_t)sg.slot * rows_b + r_out] = lse_v;
+                }
+                tc_fence_before();
+            }
+        }
+        __syncthreads();
+        if (!more_sh || abort_sh) break;
+        __syncthreads();
+    }
+
+    if (warp == 1 && lane == 0) {
+        volatile int never = 0;
+        umma_commit(&end_bar);
+        mbar_wait_one(&end_bar, 0, &never, nullptr, lim_ns);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // the peer no longer writes into this CTA's shared memory
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+uint32_t mla_pair_fixed_smem() { return P_QBYTES + P_XBYTES; }
+uint32_t mla_pair_stage_bytes() { return P_STAGE; }
+
+cudaError_t launch_mla_pair(const CUtensorMap &qm, const CUtensorMap &qrm, const CUtensorMap &lm,
+                            const CUtensorMap &rm, const LatentArgs &a, int grid, size_t smem, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(mla_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    mla_pair_kernel<<<grid, 384, smem, st>>>(qm, qrm, lm, rm, a);
+    return cudaGetLastError();
+}
+
+}  // namespace kvd
