@@ -88,6 +88,22 @@ def committed_traffic(kind, workload, qlen):
     return None
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(vals, dist=None, device="cpu"):
+    """Each value's maximum over all ranks: a replica step is as slow as the slowest GPU."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    import torch
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def aggregate(step_us, kv_bytes, world):
+    """Whole-job KV throughput of `world` replicas that each moved kv_bytes in step_us (max over ranks)."""
+    return world * kv_bytes / (step_us * 1e-6) / 1e9
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi clock/throttle samples for one GPU while the timed region runs."""
@@ -354,10 +370,7 @@ def main():
     t_step = statistics.mean(step_ms)
     t_kern = statistics.mean(kern_ms)
     t_e2e = statistics.mean(e2e_ms)
-    if pg is not None:
-        v = torch.tensor([t_step, t_kern, t_e2e], dtype=torch.float64, device=dev)
-        pg.all_reduce(v, op=pg.ReduceOp.MAX)
-        t_step, t_kern, t_e2e = (float(x) for x in v.tolist())
+    t_step, t_kern, t_e2e = max_over_ranks([t_step, t_kern, t_e2e], pg, device=dev)
 
     hbm, tfl, peak_src = load_peaks()
     variant_kind = "latent" if inp.variant == "gla" else "group"
@@ -374,7 +387,7 @@ def main():
     roof["traffic"] = committed_traffic(variant_kind, args.workload, inp.L)
     roof["roofline_us"] = accounting.roofline_us(nbytes, flops, hbm, tfl)
 
-    kv_gbs = kvb / (t_step * 1e-3) / 1e9
+    kv_gbs = aggregate(t_step * 1e3, kvb, 1)
     line = {"metric": METRIC, "value": t_step * 1e3, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": t_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
