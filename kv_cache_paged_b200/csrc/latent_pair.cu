@@ -12,9 +12,12 @@
 // for bit), run the same softmax and accumulate O for their own 256 latent columns, which are
 // exactly the latent columns they loaded.  Every byte of the cache is read once per pair.
 //
-// Roles per CTA: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4..11 softmax
-// (two threads per row, one per 32-token half of the tile).  Tensor memory: O [0, 256),
-// two partial-S buffers [256, 384), two P buffers [384, 448).  Every wait is bounded.
+// Roles per CTA: warps 0..3 exchange (one per TMEM lane quadrant: load the partial S of a
+// tile, send it, add the peer's and write the full S back into tensor memory), warps 4..11
+// softmax (two threads per row, one per 32-token half of the tile), warp 12 TMA producer,
+// warp 13 MMA issuer (one thread).  S is triple-buffered so that the exchange of tile j+1
+// overlaps the softmax of tile j.  Tensor memory: O [0, 256), three S buffers [256, 448),
+// two P buffers [448, 512).  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -32,16 +35,19 @@ constexpr uint32_t P_QBYTES = P_QLAT + 128 * 64;          // + rope half: 128 ro
 constexpr uint32_t P_CHUNK = PTOK * 128;                  // one 64-dim chunk of a tile
 constexpr uint32_t P_STAGE = 4 * P_CHUNK + PTOK * 64;     // latent half + rope half
 constexpr uint32_t P_XBYTES = 128 * 64 * 4;               // the peer's partial S (fp32)
-constexpr uint32_t P_SCOL = PDV, P_PCOL = PDV + 2 * PTOK, P_PCOLS = PTOK / 2;
+constexpr int P_NSB = 3;                                  // S buffers
+constexpr uint32_t P_SCOL = PDV, P_PCOL = PDV + P_NSB * PTOK, P_PCOLS = PTOK / 2;
+constexpr int W_PROD = 12, W_MMA = 13;
 constexpr float P_RESCALE_LOG2 = 8.f;
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     mla_pair_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap qrmap,
                     const __grid_constant__ CUtensorMap latmap, const __grid_constant__ CUtensorMap ropemap,
                     const LatentArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
-    __shared__ uint64_t qfull_bar, qempty_bar, sfull_bar[2], sfree_bar[2], pfull_bar[2], pfree_bar[2], end_bar;
+    __shared__ uint64_t qfull_bar, qempty_bar, pfull_bar[2], pfree_bar[2], end_bar;
+    __shared__ uint64_t sfull_bar[P_NSB], sready_bar[P_NSB], sfree_bar[P_NSB];
     __shared__ uint64_t xbar, xfull_bar, xfree_bar;
     __shared__ Seg segs[PMAXSEG];
     __shared__ int nseg_sh, more_sh;
@@ -75,23 +81,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         mbar_init(&qfull_bar, 1);
         mbar_init(&qempty_bar, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&sfull_bar[s], 1);
-            mbar_init(&sfree_bar[s], 8);
             mbar_init(&pfull_bar[s], 8);
             mbar_init(&pfree_bar[s], 1);
+        }
+        for (int s = 0; s < P_NSB; ++s) {
+            mbar_init(&sfull_bar[s], 1);    // partial S computed (MMA commit)
+            mbar_init(&sready_bar[s], 4);   // full S written back (exchange warps)
+            mbar_init(&sfree_bar[s], 8);    // full S read (softmax warps)
         }
         mbar_init(&end_bar, 1);
         mbar_init(&xbar, 8);
         // xfull: one local arrival that arms the expected bytes, completed by the peer's st.async
-        // (32 KB per tile); xfree: one arrival from each of the peer's 8 softmax warps
+        // (32 KB per tile); xfree: one arrival from each of the peer's 4 exchange warps
         mbar_init(&xfull_bar, 1);
-        mbar_init(&xfree_bar, 8);
+        mbar_init(&xfree_bar, 4);
         mbar_arrive_expect_tx(&xfull_bar, P_XBYTES);  // arm the first tile's exchange
         abort_sh = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(&tmem_sh, 512);
-    if (warp == 0 && lane == 0) {
+    if (warp == W_MMA) tmem_alloc(&tmem_sh, 512);
+    if (warp == W_PROD && lane == 0) {
         tma_prefetch_desc(&qmap);
         tma_prefetch_desc(&qrmap);
         tma_prefetch_desc(&latmap);
@@ -105,10 +114,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 
     uint32_t p_issued = 0, p_qloads = 0;
     uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;
-    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0, x_p = 0;
+    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0;   // softmax
+    uint32_t e_t = 0;                                   // exchange
 
     for (int skip = 0;; skip += PMAXSEG) {
-        if (warp == 0) {
+        if (warp == W_PROD) {
             int cnt = 0;
             plan_walk(a.seqlens, a.B, PTOK, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
                 if (cnt >= skip && cnt < skip + PMAXSEG) segs[cnt - skip] = s;
@@ -122,7 +132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         __syncthreads();
         const int nseg = nseg_sh;
 
-        if (warp == 0) {
+        if (warp == W_PROD) {
             // ================================================================ producer
             const uint64_t pol = policy_evict_first();
             bool stop = false;
@@ -188,7 +198,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                     mbar_wait_warp(&full_bar[k % nstage], (k / nstage) & 1, &never, nullptr, lim_ns);
                 if (p_qloads) mbar_wait_warp(&qfull_bar, (p_qloads - 1) & 1, &never, nullptr, lim_ns);
             }
-        } else if (warp == 1) {
+        } else if (warp == W_MMA) {
             // ================================================================ MMA issuer
             if (lane == 0) {
                 constexpr uint32_t idesc_s = umma_idesc_bf16(128, PTOK, false, false);
@@ -200,8 +210,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                 auto issue_s = [&](uint32_t gt) -> bool {
                     const uint32_t stage = gt % nstage;
                     if (!mbar_wait_one(&full_bar[stage], (gt / nstage) & 1, &abort_sh, a.err, lim_ns)) return false;
-                    const uint32_t sb = m_s & 1;
-                    if (!mbar_wait_one(&sfree_bar[sb], ((m_s >> 1) & 1) ^ 1, &abort_sh, a.err, lim_ns)) return false;
+                    const uint32_t sb = m_s % P_NSB;
+                    if (!mbar_wait_one(&sfree_bar[sb], ((m_s / P_NSB) & 1) ^ 1, &abort_sh, a.err, lim_ns)) return false;
                     tc_fence_after();
                     const uint32_t d = tmem + P_SCOL + sb * PTOK;
                     const uint64_t dk0 = umma_desc(st0 + stage * P_STAGE, 16, 1024, 2);
@@ -255,7 +265,82 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                 }
             }
             __syncwarp();
-        } else if (warp >= 4) {
+        } else if (warp < 4) {
+            // ================================================================ exchange
+            // thread = row; the whole 64-token partial S row goes to the peer, the peer's
+            // comes back, and the sum replaces the partial in tensor memory
+            const int r = warp * 32 + lane;
+            const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+            const uint32_t x_row = smem_u32(xbuf_s) + r * 256;
+            const uint32_t x_row_peer = mapa_shared(x_row, peer);
+            const uint32_t peer_xfull = mapa_shared(smem_u32(&xfull_bar), peer);
+            const uint32_t peer_xfree = mapa_shared(smem_u32(&xfree_bar), peer);
+            bool ok = true;
+            for (int si = 0; si < nseg && ok; ++si) {
+                const int n = segs[si].t1 - segs[si].t0;
+                for (int j = 0; j < n; ++j, ++e_t) {
+                    const uint32_t sb = e_t % P_NSB;
+                    if (!mbar_wait_warp(&sfull_bar[sb], (e_t / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = tmem + lane_base + P_SCOL + sb * PTOK;
+                    float sp[PTOK];
+                    {
+                        float t32[32];
+                        tmem_ld32(sa, t32);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) sp[k] = t32[k];
+                        tmem_ld32(sa + 32, t32);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) sp[32 + k] = t32[k];
+                    }
+                    // the peer has read what this CTA sent for the previous tile
+                    if (e_t > 0 && !mbar_wait_warp_cluster(&xfree_bar, (e_t - 1) & 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int c16 = 0; c16 < 16; ++c16)
+                        st_async_v4(x_row_peer + ((c16 ^ (r & 15)) << 4), sp[4 * c16], sp[4 * c16 + 1],
+                                    sp[4 * c16 + 2], sp[4 * c16 + 3], peer_xfull);
+                    if (!mbar_wait_warp_cluster(&xfull_bar, e_t & 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int c16 = 0; c16 < 16; ++c16) {
+                        float4 v;
+                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                                     : "r"(x_row + ((c16 ^ (r & 15)) << 4))
+                                     : "memory");
+                        sp[4 * c16] += v.x;
+                        sp[4 * c16 + 1] += v.y;
+                        sp[4 * c16 + 2] += v.z;
+                        sp[4 * c16 + 3] += v.w;
+                    }
+                    // this warp's rows are read: arm the next exchange and free the buffer
+                    __syncwarp();
+                    if (threadIdx.x == 0) mbar_arrive_expect_tx(&xfull_bar, P_XBYTES);
+                    if (lane == 0) mbar_arrive_cluster(peer_xfree);
+                    {
+                        float t32[32];
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) t32[k] = sp[k];
+                        tmem_st32(sa, t32);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) t32[k] = sp[32 + k];
+                        tmem_st32(sa + 32, t32);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sready_bar[sb]);
+                }
+            }
+        } else if (warp >= 4 && warp < 12) {
             // ================================================================ softmax / epilogue
             constexpr int HC = PTOK / 2;
             const int st_id = threadIdx.x - 128;
@@ -267,11 +352,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
             const bool warp_live = rt * 128 + (warp & 3) * 32 < R;
             const int i_row = row_ok ? n_row / g : 0;
             const int head = row_ok ? c * g + n_row % g : 0;
-            // my row of the exchange buffer, as this CTA and as the peer addresses it
-            const uint32_t x_row = smem_u32(xbuf_s) + r * 256;
-            const uint32_t x_row_peer = mapa_shared(x_row, peer);
-            const uint32_t peer_xfull = mapa_shared(smem_u32(&xfull_bar), peer);
-            const uint32_t peer_xfree = mapa_shared(smem_u32(&xfree_bar), peer);
             bool ok = true;
             auto wait_pv = [&](uint32_t k) -> bool {
                 return mbar_wait_warp(&pfree_bar[k & 1], (k >> 1) & 1, &abort_sh, a.err, lim_ns);
@@ -294,8 +374,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                 float m_ref = -INFINITY, l = 0.f, lq = 0.f;
                 for (int tile = sg.t0; tile < sg.t1; ++tile) {
                     const int tok0 = tile * PTOK + hf * HC;
-                    const uint32_t sb = x_s & 1;
-                    if (!mbar_wait_warp(&sfull_bar[sb], (x_s >> 1) & 1, &abort_sh, a.err, lim_ns)) {
+                    const uint32_t sb = x_s % P_NSB;
+                    if (!mbar_wait_warp(&sready_bar[sb], (x_s / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
                         ok = false;
                         break;
                     }
@@ -306,41 +386,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sfree_bar[sb]);
                     ++x_s;
-
-                    // ---- swap partial scores with the peer CTA (fp32, distributed shared memory)
-                    if (x_p > 0 && !mbar_wait_warp_cluster(&xfree_bar, (x_p - 1) & 1, &abort_sh, a.err, lim_ns)) {
-                        ok = false;
-                        break;
-                    }
-#pragma unroll
-                    for (int c4 = 0; c4 < HC / 4; ++c4) {
-                        const uint32_t c16 = hf * (HC / 4) + c4;
-                        st_async_v4(x_row_peer + ((c16 ^ (r & 15)) << 4), s[4 * c4], s[4 * c4 + 1], s[4 * c4 + 2],
-                                    s[4 * c4 + 3], peer_xfull);
-                    }
-                    if (!mbar_wait_warp_cluster(&xfull_bar, x_p & 1, &abort_sh, a.err, lim_ns)) {
-                        ok = false;
-                        break;
-                    }
-#pragma unroll
-                    for (int c4 = 0; c4 < HC / 4; ++c4) {
-                        const uint32_t c16 = hf * (HC / 4) + c4;
-                        float4 v;
-                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                                     : "r"(x_row + ((c16 ^ (r & 15)) << 4))
-                                     : "memory");
-                        s[4 * c4] += v.x;
-                        s[4 * c4 + 1] += v.y;
-                        s[4 * c4 + 2] += v.z;
-                        s[4 * c4 + 3] += v.w;
-                    }
-                    // this warp's rows are read (the sums above used them): arm the next exchange,
-                    // then let the peer overwrite the buffer
-                    __syncwarp();
-                    if (threadIdx.x == 128) mbar_arrive_expect_tx(&xfull_bar, P_XBYTES);
-                    if (lane == 0) mbar_arrive_cluster(peer_xfree);
-                    ++x_p;
 
                     float mx = -INFINITY;
                     if (warp_live) {
@@ -494,7 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         __syncthreads();
     }
 
-    if (warp == 1 && lane == 0) {
+    if (warp == W_MMA && lane == 0) {
         volatile int never = 0;
         umma_commit(&end_bar);
         mbar_wait_one(&end_bar, 0, &never, nullptr, lim_ns);
@@ -503,7 +548,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     __syncthreads();
     cluster_sync();  // the peer no longer writes into this CTA's shared memory
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (warp == W_MMA) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace
@@ -515,7 +560,7 @@ cudaError_t launch_mla_pair(const CUtensorMap &qm, const CUtensorMap &qrm, const
                             const CUtensorMap &rm, const LatentArgs &a, int grid, size_t smem, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(mla_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    mla_pair_kernel<<<grid, 384, smem, st>>>(qm, qrm, lm, rm, a);
+    mla_pair_kernel<<<grid, 448, smem, st>>>(qm, qrm, lm, rm, a);
     return cudaGetLastError();
 }
 
