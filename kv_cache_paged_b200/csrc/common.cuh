@@ -487,5 +487,16 @@ __device__ __forceinline__ void st_async_v4(uint32_t caddr, float a, float b, fl
                  "f"(a), "f"(b), "f"(c), "f"(d), "r"(caddr_bar)
                  : "memory");
 }
+// Bulk copy (the async copy engine) of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) from this CTA's shared memory to another CTA's; completes `bytes` of the
+// transaction count of the destination CTA's mbarrier at caddr_bar.  The source may be
+// rewritten once that mbarrier's phase has completed.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t caddr_dst, uint32_t saddr_src, uint32_t bytes,
+                                                  uint32_t caddr_bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     caddr_dst),
+                 "r"(saddr_src), "r"(bytes), "r"(caddr_bar)
+                 : "memory");
+}
 }  // namespace kvd
 #endif  // __CUDACC__

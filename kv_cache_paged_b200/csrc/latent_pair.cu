@@ -12,12 +12,13 @@
 // for bit), run the same softmax and accumulate O for their own 256 latent columns, which are
 // exactly the latent columns they loaded.  Every byte of the cache is read once per pair.
 //
-// Roles per CTA: warps 0..3 exchange (one per TMEM lane quadrant: load the partial S of a
-// tile, send it, add the peer's and write the full S back into tensor memory), warps 4..11
-// softmax (two threads per row, one per 32-token half of the tile), warp 12 TMA producer,
-// warp 13 MMA issuer (one thread).  S is triple-buffered so that the exchange of tile j+1
-// overlaps the softmax of tile j.  Tensor memory: O [0, 256), three S buffers [256, 448),
-// two P buffers [448, 512).  Every wait is bounded.
+// Roles per CTA: warps 0..3 send (one per TMEM lane quadrant: load this CTA's partial S of a
+// tile and store it into the peer's receive buffer), warps 4..11 softmax (two threads per row,
+// one per 32-token half of the tile; each adds the peer's partial from its receive buffer to its
+// own from tensor memory), warp 12 TMA producer, warp 13 MMA issuer (one thread).  S is
+// triple-buffered and the receive buffer double-buffered, so the transfer of tile j+1 overlaps
+// the softmax of tile j.  Tensor memory: O [0, 256), three S buffers [256, 448), two P buffers
+// [448, 512).  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -34,7 +35,8 @@ constexpr uint32_t P_QLAT = 4 * 16384;                    // q latent half: 4 ch
 constexpr uint32_t P_QBYTES = P_QLAT + 128 * 64;          // + rope half: 128 rows x 64 B
 constexpr uint32_t P_CHUNK = PTOK * 128;                  // one 64-dim chunk of a tile
 constexpr uint32_t P_STAGE = 4 * P_CHUNK + PTOK * 64;     // latent half + rope half
-constexpr uint32_t P_XBYTES = 128 * 64 * 4;               // the peer's partial S (fp32)
+constexpr uint32_t P_XHALF = 128 * 32 * 4;               // one 32-token half of a partial S tile (fp32)
+constexpr uint32_t P_XBYTES = 4 * P_XHALF;                // send and receive buffers, one per half
 constexpr int P_NSB = 3;                                  // S buffers
 constexpr uint32_t P_SCOL = PDV, P_PCOL = PDV + P_NSB * PTOK, P_PCOLS = PTOK / 2;
 constexpr int W_PROD = 12, W_MMA = 13;
@@ -47,8 +49,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
     __shared__ uint64_t qfull_bar, qempty_bar, pfull_bar[2], pfree_bar[2], end_bar;
-    __shared__ uint64_t sfull_bar[P_NSB], sready_bar[P_NSB], sfree_bar[P_NSB];
-    __shared__ uint64_t xbar, xfull_bar, xfree_bar;
+    __shared__ uint64_t sfull_bar[P_NSB], sfree_bar[P_NSB];
+    __shared__ uint64_t xbar, xfull_bar[2], xfree_bar[2];
     __shared__ Seg segs[PMAXSEG];
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
@@ -57,8 +59,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
 
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *q_s = smem;
-    uint8_t *xbuf_s = smem + P_QBYTES;                      // receives the peer's partial S
-    uint8_t *stage_s = xbuf_s + P_XBYTES;
+    uint8_t *send_s = smem + P_QBYTES;                      // this CTA's partial S, per half
+    uint8_t *recv_s = send_s + 2 * P_XHALF;                 // the peer's partial S, per half
+    uint8_t *stage_s = send_s + P_XBYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t kr = cluster_rank();                     // 0 or 1: which half of the key
@@ -86,16 +89,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         }
         for (int s = 0; s < P_NSB; ++s) {
             mbar_init(&sfull_bar[s], 1);    // partial S computed (MMA commit)
-            mbar_init(&sready_bar[s], 4);   // full S written back (exchange warps)
-            mbar_init(&sfree_bar[s], 8);    // full S read (softmax warps)
+            mbar_init(&sfree_bar[s], 12);   // partial S read by the 4 send and 8 softmax warps
         }
         mbar_init(&end_bar, 1);
         mbar_init(&xbar, 8);
-        // xfull: one local arrival that arms the expected bytes, completed by the peer's st.async
-        // (32 KB per tile); xfree: one arrival from each of the peer's 4 exchange warps
-        mbar_init(&xfull_bar, 1);
-        mbar_init(&xfree_bar, 4);
-        mbar_arrive_expect_tx(&xfull_bar, P_XBYTES);  // arm the first tile's exchange
+        // per 32-token half h of a tile: xfull[h] takes one local arrival that arms the expected
+        // bytes and is completed by the peer's bulk copies (16 KB); xfree[h] takes one arrival
+        // from each of the peer's 4 softmax warps that read half h
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&xfull_bar[h], 1);
+            mbar_init(&xfree_bar[h], 4);
+            mbar_arrive_expect_tx(&xfull_bar[h], P_XHALF);  // armed for the first tile
+        }
         abort_sh = 0;
         fence_mbar_init();
     }
@@ -115,7 +120,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     uint32_t p_issued = 0, p_qloads = 0;
     uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;
     uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0;   // softmax
-    uint32_t e_t = 0;                                   // exchange
+    uint32_t e_t = 0;                                   // send
 
     for (int skip = 0;; skip += PMAXSEG) {
         if (warp == W_PROD) {
@@ -266,19 +271,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
             }
             __syncwarp();
         } else if (warp < 4) {
-            // ================================================================ exchange
-            // thread = row; the whole 64-token partial S row goes to the peer, the peer's
-            // comes back, and the sum replaces the partial in tensor memory
+            // ================================================================ send
+            // thread = row.  Each 32-token half of the row's partial S is staged in this CTA's
+            // send buffer (16-byte chunks XOR-swizzled by row), then one bulk copy per warp and
+            // half moves the warp's 32 rows (4 KB) into the peer's receive buffer.
             const int r = warp * 32 + lane;
             const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-            const uint32_t x_row = smem_u32(xbuf_s) + r * 256;
-            const uint32_t x_row_peer = mapa_shared(x_row, peer);
-            const uint32_t peer_xfull = mapa_shared(smem_u32(&xfull_bar), peer);
-            const uint32_t peer_xfree = mapa_shared(smem_u32(&xfree_bar), peer);
+            const uint32_t peer_recv = mapa_shared(smem_u32(recv_s), peer);
+            const uint32_t peer_xfull[2] = {mapa_shared(smem_u32(&xfull_bar[0]), peer),
+                                            mapa_shared(smem_u32(&xfull_bar[1]), peer)};
             bool ok = true;
             for (int si = 0; si < nseg && ok; ++si) {
                 const int n = segs[si].t1 - segs[si].t0;
-                for (int j = 0; j < n; ++j, ++e_t) {
+                for (int j = 0; j < n && ok; ++j, ++e_t) {
                     const uint32_t sb = e_t % P_NSB;
                     if (!mbar_wait_warp(&sfull_bar[sb], (e_t / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
                         ok = false;
@@ -286,58 +291,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                     }
                     tc_fence_after();
                     const uint32_t sa = tmem + lane_base + P_SCOL + sb * PTOK;
-                    float sp[PTOK];
-                    {
-                        float t32[32];
-                        tmem_ld32(sa, t32);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) sp[k] = t32[k];
-                        tmem_ld32(sa + 32, t32);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) sp[32 + k] = t32[k];
-                    }
-                    // the peer has read what this CTA sent for the previous tile
-                    if (e_t > 0 && !mbar_wait_warp_cluster(&xfree_bar, (e_t - 1) & 1, &abort_sh, a.err, lim_ns)) {
-                        ok = false;
-                        break;
-                    }
-#pragma unroll
-                    for (int c16 = 0; c16 < 16; ++c16)
-                        st_async_v4(x_row_peer + ((c16 ^ (r & 15)) << 4), sp[4 * c16], sp[4 * c16 + 1],
-                                    sp[4 * c16 + 2], sp[4 * c16 + 3], peer_xfull);
-                    if (!mbar_wait_warp_cluster(&xfull_bar, e_t & 1, &abort_sh, a.err, lim_ns)) {
-                        ok = false;
-                        break;
-                    }
-#pragma unroll
-                    for (int c16 = 0; c16 < 16; ++c16) {
-                        float4 v;
-                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                     : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                                     : "r"(x_row + ((c16 ^ (r & 15)) << 4))
-                                     : "memory");
-                        sp[4 * c16] += v.x;
-                        sp[4 * c16 + 1] += v.y;
-                        sp[4 * c16 + 2] += v.z;
-                        sp[4 * c16 + 3] += v.w;
-                    }
-                    // this warp's rows are read: arm the next exchange and free the buffer
-                    __syncwarp();
-                    if (threadIdx.x == 0) mbar_arrive_expect_tx(&xfull_bar, P_XBYTES);
-                    if (lane == 0) mbar_arrive_cluster(peer_xfree);
-                    {
-                        float t32[32];
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) t32[k] = sp[k];
-                        tmem_st32(sa, t32);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) t32[k] = sp[32 + k];
-                        tmem_st32(sa + 32, t32);
-                    }
-                    tmem_st_wait();
+                    float sp[2][32];
+                    tmem_ld32(sa, sp[0]);
+                    tmem_ld32(sa + 32, sp[1]);
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sready_bar[sb]);
+                    if (lane == 0) mbar_arrive(&sfree_bar[sb]);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        // the peer has read the previous tile's half h, so both this CTA's send
+                        // buffer (the copy's source) and the peer's receive buffer are free
+                        if (e_t > 0 &&
+                            !mbar_wait_warp_cluster(&xfree_bar[h], (e_t - 1) & 1, &abort_sh, a.err, lim_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t row = smem_u32(send_s + h * P_XHALF) + r * 128;
+#pragma unroll
+                        for (int c8 = 0; c8 < 8; ++c8)
+                            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((c8 ^ (r & 7)) << 4)),
+                                         "f"(sp[h][4 * c8]), "f"(sp[h][4 * c8 + 1]), "f"(sp[h][4 * c8 + 2]),
+                                         "f"(sp[h][4 * c8 + 3])
+                                         : "memory");
+                        fence_proxy_async();
+                        __syncwarp();
+                        if (lane == 0)
+                            bulk_copy_to_peer(peer_recv + h * P_XHALF + warp * 4096,
+                                              smem_u32(send_s + h * P_XHALF) + warp * 4096, 4096, peer_xfull[h]);
+                    }
                 }
             }
         } else if (warp >= 4 && warp < 12) {
@@ -350,6 +331,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
             const int n_row = rt * 128 + r;
             const bool row_ok = n_row < R;
             const bool warp_live = rt * 128 + (warp & 3) * 32 < R;
+            const uint32_t peer_xfree[2] = {mapa_shared(smem_u32(&xfree_bar[0]), peer),
+                                                mapa_shared(smem_u32(&xfree_bar[1]), peer)};
             const int i_row = row_ok ? n_row / g : 0;
             const int head = row_ok ? c * g + n_row % g : 0;
             bool ok = true;
@@ -375,7 +358,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                 for (int tile = sg.t0; tile < sg.t1; ++tile) {
                     const int tok0 = tile * PTOK + hf * HC;
                     const uint32_t sb = x_s % P_NSB;
-                    if (!mbar_wait_warp(&sready_bar[sb], (x_s / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
+                    if (!mbar_wait_warp(&sfull_bar[sb], (x_s / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
                         ok = false;
                         break;
                     }
@@ -385,6 +368,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sfree_bar[sb]);
+                    // S = own partial + the peer's (the peer adds in the opposite order; fp32
+                    // addition commutes, so both CTAs see the same S bit for bit)
+                    if (!mbar_wait_warp_cluster(&xfull_bar[hf], x_s & 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    // the phase is complete: arm the next tile's before any warp releases the buffer
+                    if (threadIdx.x == 128 + 128 * hf) mbar_arrive_expect_tx(&xfull_bar[hf], P_XHALF);
+                    {
+                        const uint32_t row = smem_u32(recv_s + hf * P_XHALF) + r * 128;
+#pragma unroll
+                        for (int c8 = 0; c8 < 8; ++c8) {
+                            float4 v;
+                            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                         : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                                         : "r"(row + ((c8 ^ (r & 7)) << 4))
+                                         : "memory");
+                            s[4 * c8] += v.x;
+                            s[4 * c8 + 1] += v.y;
+                            s[4 * c8 + 2] += v.z;
+                            s[4 * c8 + 3] += v.w;
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(peer_xfree[hf]);
                     ++x_s;
 
                     float mx = -INFINITY;
