@@ -5,20 +5,21 @@
 // columns alone fills tensor memory, so the value columns are split over two CTAs.  Rather
 // than have both CTAs compute the same 128 x 576 score product, the pair (a thread-block
 // cluster of 2) splits the 576-wide key dimension as well: CTA k holds q's latent dims
-// [256k, 256k + 256) and rope dims [32k, 32k + 32) (72 KB of shared memory instead of 144 KB),
+// [256k, 256k + 256) and rope dims [32k, 32k + 32),
 // loads only those columns of each 64-token tile (36 KB), computes a partial score
 // S_k = Q_k K_k^T on tcgen05 and swaps it with its peer through distributed shared memory.
 // Both CTAs then hold the same S = S_0 + S_1 (fp32 addition commutes, so the sums agree bit
 // for bit), run the same softmax and accumulate O for their own 256 latent columns, which are
 // exactly the latent columns they loaded.  Every byte of the cache is read once per pair.
 //
-// Roles per CTA: warps 0..3 send (one per TMEM lane quadrant: load this CTA's partial S of a
-// tile and store it into the peer's receive buffer), warps 4..11 softmax (two threads per row,
-// one per 32-token half of the tile; each adds the peer's partial from its receive buffer to its
-// own from tensor memory), warp 12 TMA producer, warp 13 MMA issuer (one thread).  S is
-// triple-buffered and the receive buffer double-buffered, so the transfer of tile j+1 overlaps
-// the softmax of tile j.  Tensor memory: O [0, 256), three S buffers [256, 448), two P buffers
-// [448, 512).  Every wait is bounded.
+// Roles per CTA: warps 0..3 send (one per TMEM lane quadrant: write q's latent half into tensor
+// memory at the start of each sequence, then per tile load this CTA's partial S and bulk-copy it
+// into the peer's receive buffer, one 32-token half at a time), warps 4..11 softmax (two threads
+// per row, one per 32-token half of the tile; each adds the peer's partial from its receive
+// buffer to its own from tensor memory), warp 12 TMA producer, warp 13 MMA issuer (one thread).
+// Tensor memory: O [0, 256), two S buffers [256, 384) with P(j) written over S(j) as bf16 pairs,
+// and q's latent half [384, 512) as the A operand of the score product.  Keeping q there leaves
+// shared memory for four 36 KB KV stages next to the exchange buffers.  Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -31,14 +32,15 @@ namespace {
 constexpr int PMAXSEG = 32;
 constexpr int PTOK = 64;                                  // tokens per tile
 constexpr int PDV = 256;                                  // value columns per CTA
-constexpr uint32_t P_QLAT = 4 * 16384;                    // q latent half: 4 chunks x 128 rows x 128 B
-constexpr uint32_t P_QBYTES = P_QLAT + 128 * 64;          // + rope half: 128 rows x 64 B
+constexpr int P_DQK = 576;                                // q row: 512 latent + 64 rope
+constexpr uint32_t P_QBYTES = 128 * 64;                  // q rope half: 128 rows x 64 B (shared memory)
 constexpr uint32_t P_CHUNK = PTOK * 128;                  // one 64-dim chunk of a tile
 constexpr uint32_t P_STAGE = 4 * P_CHUNK + PTOK * 64;     // latent half + rope half
 constexpr uint32_t P_XHALF = 128 * 32 * 4;               // one 32-token half of a partial S tile (fp32)
 constexpr uint32_t P_XBYTES = 4 * P_XHALF;                // send and receive buffers, one per half
-constexpr int P_NSB = 3;                                  // S buffers
-constexpr uint32_t P_SCOL = PDV, P_PCOL = PDV + P_NSB * PTOK, P_PCOLS = PTOK / 2;
+constexpr int P_NSB = 2;                                  // S buffers (P is written over its S)
+constexpr uint32_t P_SCOL = PDV;                          // S buffers [256, 384)
+constexpr uint32_t P_QCOL = PDV + P_NSB * PTOK;           // q latent half [384, 512), bf16 pairs
 constexpr int W_PROD = 12, W_MMA = 13;
 constexpr float P_RESCALE_LOG2 = 8.f;
 
@@ -48,8 +50,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                     const LatentArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
-    __shared__ uint64_t qfull_bar, qempty_bar, pfull_bar[2], pfree_bar[2], end_bar;
-    __shared__ uint64_t sfull_bar[P_NSB], sfree_bar[P_NSB];
+    __shared__ uint64_t qfull_bar, qtm_bar, qempty_bar, pfull_bar[P_NSB], pfree_bar[P_NSB], end_bar;
+    __shared__ uint64_t sfull_bar[P_NSB], sread_bar[P_NSB];
     __shared__ uint64_t xbar, xfull_bar[2], xfree_bar[2];
     __shared__ Seg segs[PMAXSEG];
     __shared__ int nseg_sh, more_sh;
@@ -81,7 +83,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(&qfull_bar, 1);
+        mbar_init(&qfull_bar, 1);   // q rope half (TMA)
+        mbar_init(&qtm_bar, 4);     // q latent half written into tensor memory by the send warps
         mbar_init(&qempty_bar, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&pfull_bar[s], 8);
@@ -89,7 +92,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         }
         for (int s = 0; s < P_NSB; ++s) {
             mbar_init(&sfull_bar[s], 1);    // partial S computed (MMA commit)
-            mbar_init(&sfree_bar[s], 12);   // partial S read by the 4 send and 8 softmax warps
+            mbar_init(&sread_bar[s], 4);    // partial S read by the send warps (P may overwrite it)
         }
         mbar_init(&end_bar, 1);
         mbar_init(&xbar, 8);
@@ -106,7 +109,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     }
     if (warp == W_MMA) tmem_alloc(&tmem_sh, 512);
     if (warp == W_PROD && lane == 0) {
-        tma_prefetch_desc(&qmap);
         tma_prefetch_desc(&qrmap);
         tma_prefetch_desc(&latmap);
         tma_prefetch_desc(&ropemap);
@@ -118,9 +120,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     const uint32_t tmem = tmem_sh;
 
     uint32_t p_issued = 0, p_qloads = 0;
-    uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;
+    uint32_t m_tile = 0, m_q = 0;
     uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0;   // softmax
-    uint32_t e_t = 0;                                   // send
+    uint32_t e_t = 0, e_q = 0;                          // send
 
     for (int skip = 0;; skip += PMAXSEG) {
         if (warp == W_PROD) {
@@ -150,15 +152,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                     break;
                 }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&qfull_bar, (uint32_t)rows_tile * (4 * 128 + 64));
+                    mbar_arrive_expect_tx(&qfull_bar, (uint32_t)rows_tile * 64);
                     for (int run = 0; run * rb < rows_tile; ++run) {
                         const int n0 = rt * 128 + run * rb;
                         const int i = n0 / g, h0 = n0 % g;
                         const int row = (sg.b * a.L + i) * a.h_q + c * g + h0;
-                        for (int ch = 0; ch < 4; ++ch)
-                            tma_load_3d(q_s + ch * 16384 + run * rb * 128, &qmap, &qfull_bar, 0, row, 4 * kr + ch,
-                                        pol);
-                        tma_load_3d(q_s + P_QLAT + run * rb * 64, &qrmap, &qfull_bar, 0, row, 16 + kr, pol);
+                        tma_load_3d(q_s + run * rb * 64, &qrmap, &qfull_bar, 0, row, 16 + kr, pol);
                     }
                 }
                 ++p_qloads;
@@ -209,34 +208,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                 constexpr uint32_t idesc_s = umma_idesc_bf16(128, PTOK, false, false);
                 constexpr uint32_t idesc_pv = umma_idesc_bf16(128, PDV, false, true);
                 const uint32_t st0 = smem_u32(stage_s);
-                const uint64_t dq0 = umma_desc(smem_u32(q_s), 16, 1024, 2);          // latent, 128 B swizzle
-                const uint64_t dqr = umma_desc(smem_u32(q_s) + P_QLAT, 16, 512, 4);  // rope half, 64 B swizzle
+                const uint64_t dqr = umma_desc(smem_u32(q_s), 16, 512, 4);  // rope half, 64 B swizzle
                 bool ok = true;
+                // S(j) goes into buffer j % 2, where P(j - 2) was: the MMAs of one thread run in
+                // issue order, so the score product of tile j, issued after the P.V product of
+                // tile j - 2, cannot overwrite that P before it is read
                 auto issue_s = [&](uint32_t gt) -> bool {
                     const uint32_t stage = gt % nstage;
                     if (!mbar_wait_one(&full_bar[stage], (gt / nstage) & 1, &abort_sh, a.err, lim_ns)) return false;
-                    const uint32_t sb = m_s % P_NSB;
-                    if (!mbar_wait_one(&sfree_bar[sb], ((m_s / P_NSB) & 1) ^ 1, &abort_sh, a.err, lim_ns)) return false;
                     tc_fence_after();
-                    const uint32_t d = tmem + P_SCOL + sb * PTOK;
+                    const uint32_t d = tmem + P_SCOL + (gt % P_NSB) * PTOK;
                     const uint64_t dk0 = umma_desc(st0 + stage * P_STAGE, 16, 1024, 2);
                     const uint64_t dkr = umma_desc(st0 + stage * P_STAGE + 4 * P_CHUNK, 16, 512, 4);
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(d, dq0 + (uint64_t)((ch * 16384 + kk * 32) >> 4),
-                                      dk0 + (uint64_t)((ch * P_CHUNK + kk * 32) >> 4), idesc_s, (ch | kk) != 0);
+                            umma_bf16_ts(d, tmem + P_QCOL + ch * 32 + kk * 8,
+                                         dk0 + (uint64_t)((ch * P_CHUNK + kk * 32) >> 4), idesc_s, (ch | kk) != 0);
 #pragma unroll
                     for (int kk = 0; kk < 2; ++kk)
                         umma_bf16(d, dqr + (uint64_t)(kk * 2), dkr + (uint64_t)(kk * 2), idesc_s, 1u);
-                    umma_commit(&sfull_bar[sb]);
-                    ++m_s;
+                    umma_commit(&sfull_bar[gt % P_NSB]);
                     return true;
                 };
                 for (int si = 0; si < nseg && ok; ++si) {
                     const int n = segs[si].t1 - segs[si].t0;
                     if (!mbar_wait_one(&qfull_bar, m_q & 1, &abort_sh, a.err, lim_ns)) break;
+                    if (!mbar_wait_one(&qtm_bar, m_q & 1, &abort_sh, a.err, lim_ns)) break;
                     ++m_q;
                     tc_fence_after();
                     if (!issue_s(m_tile)) break;
@@ -247,24 +246,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                                 ok = false;
                                 break;
                             }
-                            if (j + 1 == n - 1) umma_commit(&qempty_bar);
+                            if (j + 1 == n - 1) umma_commit(&qempty_bar);  // q is free once these finish
                         }
-                        const uint32_t pb = m_pv & 1;
-                        if (!mbar_wait_one(&pfull_bar[pb], (m_pv >> 1) & 1, &abort_sh, a.err, lim_ns)) {
+                        const uint32_t pb = (m_tile + j) % P_NSB;
+                        if (!mbar_wait_one(&pfull_bar[pb], ((m_tile + j) / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         const uint32_t stage = (m_tile + j) % nstage;
                         const uint64_t dv0 = umma_desc(st0 + stage * P_STAGE, P_CHUNK, 1024, 2);
-                        const uint32_t pa = tmem + P_PCOL + pb * P_PCOLS;
+                        const uint32_t pa = tmem + P_SCOL + pb * PTOK;
 #pragma unroll
                         for (int kk = 0; kk < PTOK / 16; ++kk)
                             umma_bf16_ts(tmem, pa + kk * 8, dv0 + (uint64_t)(kk * 128), idesc_pv,
                                          (j > 0 || kk > 0) ? 1u : 0u);
                         umma_commit(&pfree_bar[pb]);
                         umma_commit(&empty_bar[stage]);
-                        ++m_pv;
                     }
                     m_tile += n;
                 }
@@ -280,9 +278,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
             const uint32_t peer_recv = mapa_shared(smem_u32(recv_s), peer);
             const uint32_t peer_xfull[2] = {mapa_shared(smem_u32(&xfull_bar[0]), peer),
                                             mapa_shared(smem_u32(&xfull_bar[1]), peer)};
+            const int n_row = rt * 128 + r;
             bool ok = true;
             for (int si = 0; si < nseg && ok; ++si) {
                 const int n = segs[si].t1 - segs[si].t0;
+                // q's latent half for this segment's rows goes into tensor memory (the A operand
+                // of the score product) once the previous segment's score MMAs are done with it
+                if (!mbar_wait_warp(&qempty_bar, (e_q & 1) ^ 1, &abort_sh, a.err, lim_ns)) break;
+                ++e_q;
+                tc_fence_after();
+                {
+                    const uint4 *src = nullptr;
+                    if (n_row < R) {
+                        const int i = n_row / g, h = n_row % g;
+                        src = (const uint4 *)(a.q + ((size_t)(segs[si].b * a.L + i) * a.h_q + c * g + h) * P_DQK +
+                                              kr * PDV);
+                    }
+#pragma unroll 1
+                    for (int part16 = 0; part16 < 8; ++part16) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint4 v = src ? __ldg(src + part16 * 4 + k) : make_uint4(0, 0, 0, 0);
+                            w[4 * k] = v.x;
+                            w[4 * k + 1] = v.y;
+                            w[4 * k + 2] = v.z;
+                            w[4 * k + 3] = v.w;
+                        }
+                        tmem_st16u(tmem + lane_base + P_QCOL + part16 * 16, w);
+                    }
+                    tmem_st_wait();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&qtm_bar);
                 for (int j = 0; j < n && ok; ++j, ++e_t) {
                     const uint32_t sb = e_t % P_NSB;
                     if (!mbar_wait_warp(&sfull_bar[sb], (e_t / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
@@ -296,7 +325,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                     tmem_ld32(sa + 32, sp[1]);
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sfree_bar[sb]);
+                    if (lane == 0) mbar_arrive(&sread_bar[sb]);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         // the peer has read the previous tile's half h, so both this CTA's send
@@ -342,9 +371,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
             auto exchange = [&](float v, float &other) -> bool {
                 const int buf = x_x & 1;
                 xchg_sh[buf][hf][r] = v;
+                tc_fence_before();  // this warp's tensor-memory reads happen before the arrival
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xbar);
                 if (!mbar_wait_warp(&xbar, x_x & 1, &abort_sh, a.err, lim_ns)) return false;
+                tc_fence_after();
                 other = xchg_sh[buf][hf ^ 1][r];
                 ++x_x;
                 return true;
@@ -365,9 +396,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                     tc_fence_after();
                     float s[HC];
                     tmem_ld32(tmem + lane_base + P_SCOL + sb * PTOK + hf * HC, s);
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sfree_bar[sb]);
                     // S = own partial + the peer's (the peer adds in the opposite order; fp32
                     // addition commutes, so both CTAs see the same S bit for bit)
                     if (!mbar_wait_warp_cluster(&xfull_bar[hf], x_s & 1, &abort_sh, a.err, lim_ns)) {
@@ -465,13 +493,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                             *(uint4 *)(v0 + ch * P_CHUNK + row * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                         }
                     }
-                    if (x_pv >= 2 && !wait_pv(x_pv - 2)) {
+                    // P(j) is written over S(j): both warpgroups have read their S columns (the
+                    // row-max exchange above orders that) and the send warps must have too
+                    if (!mbar_wait_warp(&sread_bar[sb], (x_pv / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     if (warp_live) {
-                        const uint32_t pa = tmem + lane_base + P_PCOL + (x_pv & 1) * P_PCOLS + hf * (HC / 2);
+                        const uint32_t pa = tmem + lane_base + P_SCOL + sb * PTOK + hf * (HC / 2);
                         uint32_t w[HC / 2];
                         float sum = 0.f;
 #pragma unroll
