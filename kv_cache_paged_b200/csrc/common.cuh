@@ -434,9 +434,12 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t caddr, float a, float b, 
     asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(caddr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
 }
-// Arrive on an mbarrier of another CTA of the cluster, releasing this thread's prior writes.
+// Arrive on an mbarrier of another CTA of the cluster (default semantics: release at CTA scope).
+// This is how a consumer hands a buffer back to a producer in the other CTA: its reads of the
+// buffer are done before the arrival.  A cluster-scope release would also wait for every earlier
+// memory operation of the thread to become visible cluster-wide, which costs thousands of cycles.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr_bar) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr_bar) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
