@@ -293,6 +293,59 @@ __device__ __forceinline__ bool mbar_wait_one(uint64_t *bar, uint32_t parity, vo
     }
 }
 
+// ----------------------------------------------------------------------------- softmax of a row slice
+// A thread holds N raw scores s[k] (fp32 q.k) of one query row for tokens tok0 + k; the row sees
+// tokens t <= lim.  c = softmax scale * log2(e), so exp(scale * s - m') = 2^(c * s - m).
+
+// max over the visible k of c * s[k] (-inf if none).  On a tile with nothing masked (`full`) the
+// raw scores are reduced first, since scaling by c is monotone (a min when c < 0).
+template <int N>
+__device__ __forceinline__ float tile_max(const float (&s)[N], bool full, int tok0, int lim, float c) {
+    if (full) {
+        float r[4] = {s[0], s[1], s[2], s[3]};
+        if (c >= 0.f) {
+#pragma unroll
+            for (int k = 4; k < N; ++k) r[k & 3] = fmaxf(r[k & 3], s[k]);
+            return fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3])) * c;
+        }
+#pragma unroll
+        for (int k = 4; k < N; ++k) r[k & 3] = fminf(r[k & 3], s[k]);
+        return fminf(fminf(r[0], r[1]), fminf(r[2], r[3])) * c;
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < N; ++k)
+        if (tok0 + k <= lim) m = fmaxf(m, s[k] * c);
+    return m;
+}
+
+// s[k] <- 2^(c * s[k] - m) for visible k and 0 elsewhere (all 0 while m = -inf: nothing visible
+// yet); returns the fp32 sum of the new s.
+template <int N>
+__device__ __forceinline__ float tile_exp(float (&s)[N], bool full, int tok0, int lim, float c, float m) {
+    if (m == -INFINITY) {
+#pragma unroll
+        for (int k = 0; k < N; ++k) s[k] = 0.f;
+        return 0.f;
+    }
+    const float nm = -m;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (full) {
+#pragma unroll
+        for (int k = 0; k < N; ++k) {
+            s[k] = ex2(fmaf(s[k], c, nm));
+            acc[k & 3] += s[k];
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < N; ++k) {
+            s[k] = tok0 + k <= lim ? ex2(fmaf(s[k], c, nm)) : 0.f;
+            acc[k & 3] += s[k];
+        }
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
 // ----------------------------------------------------------------------------- tcgen05 (5th-gen tensor cores)
 // Shared-memory matrix descriptor: start address, leading / stride byte offsets,
 // version 1 (sm_100), layout type (2 = 128-byte swizzle, 4 = 64-byte swizzle).

@@ -323,15 +323,8 @@ __global__ void __launch_bounds__(384, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&sfree_bar[sb]);
                     ++x_s;
-                    if (warp_live) {
-                        const bool full = tile * TOK + TOK - 1 <= T - a.L && row_ok;
-#pragma unroll
-                        for (int k = 0; k < HC; ++k) {
-                            const float v = (full || tok0 + k <= lim) ? s[k] * a.scale_log2 : -INFINITY;
-                            s[k] = v;
-                            mx = fmaxf(mx, v);
-                        }
-                    }
+                    const bool full = tile * TOK + TOK - 1 <= T - a.L && row_ok;  // no column masked
+                    if (warp_live) mx = tile_max(s, full, tok0, lim, a.scale_log2);
                     float mo;
                     if (!exchange(mx, mo)) {
                         ok = false;
@@ -369,18 +362,7 @@ __global__ void __launch_bounds__(384, 1)
                         }
                         tmem_st_wait();
                     }
-                    if (warp_live) {
-                        if (m_ref != -INFINITY) {
-#pragma unroll
-                            for (int k = 0; k < HC; ++k) {
-                                s[k] = ex2(s[k] - m_ref);
-                                l += s[k];
-                            }
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < HC; ++k) s[k] = 0.f;
-                        }
-                    }
+                    if (warp_live) l += tile_exp(s, full, tok0, lim, a.scale_log2, m_ref);
 
                     // tokens past T_b in this tile hold garbage: zero their value rows (P is 0 there,
                     // but 0 * NaN would still poison the product)
@@ -405,11 +387,12 @@ __global__ void __launch_bounds__(384, 1)
                     if (warp_live) {
                         const uint32_t pa = tmem + lane_base + C::P_COL + (x_pv & 1) * C::P_COLS + hf * (HC / 2);
                         uint32_t w[HC / 2];
-                        float sum = 0.f;
+                        float sum = 0.f, sum2 = 0.f;
 #pragma unroll
                         for (int k = 0; k < HC / 2; ++k) {
                             w[k] = pack_bf16(s[2 * k], s[2 * k + 1]);
-                            sum += bf16_lo(w[k]) + bf16_hi(w[k]);
+                            sum += bf16_lo(w[k]);
+                            sum2 += bf16_hi(w[k]);
                         }
                         if constexpr (HC == 32) {
                             tmem_st16u(pa, w);
@@ -417,7 +400,7 @@ __global__ void __launch_bounds__(384, 1)
                             tmem_st8u(pa, w);
                         }
                         tmem_st_wait();
-                        lq += sum;
+                        lq += sum + sum2;
                     }
                     if (ttok0 + TOK > T) fence_proxy_async();  // the zeroed value rows above
                     tc_fence_before();

@@ -424,15 +424,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                     ++x_s;
 
                     float mx = -INFINITY;
-                    if (warp_live) {
-                        const bool full = tile * PTOK + PTOK - 1 <= T - a.L && row_ok;
-#pragma unroll
-                        for (int k = 0; k < HC; ++k) {
-                            const float v = (full || tok0 + k <= lim) ? s[k] * a.scale_log2 : -INFINITY;
-                            s[k] = v;
-                            mx = fmaxf(mx, v);
-                        }
-                    }
+                    const bool full = tile * PTOK + PTOK - 1 <= T - a.L && row_ok;  // no column masked
+                    if (warp_live) mx = tile_max(s, full, tok0, lim, a.scale_log2);
                     float mo;
                     if (!exchange(mx, mo)) {
                         ok = false;
@@ -469,18 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                         }
                         tmem_st_wait();
                     }
-                    if (warp_live) {
-                        if (m_ref != -INFINITY) {
-#pragma unroll
-                            for (int k = 0; k < HC; ++k) {
-                                s[k] = ex2(s[k] - m_ref);
-                                l += s[k];
-                            }
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < HC; ++k) s[k] = 0.f;
-                        }
-                    }
+                    if (warp_live) l += tile_exp(s, full, tok0, lim, a.scale_log2, m_ref);
                     // value rows of tokens past T_b hold garbage: zero them (0 * NaN would poison O)
                     const uint32_t stage = x_tile % nstage;
                     const int ttok0 = tile * PTOK;
@@ -503,15 +485,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                     if (warp_live) {
                         const uint32_t pa = tmem + lane_base + P_SCOL + sb * PTOK + hf * (HC / 2);
                         uint32_t w[HC / 2];
-                        float sum = 0.f;
+                        float sum = 0.f, sum2 = 0.f;
 #pragma unroll
                         for (int k = 0; k < HC / 2; ++k) {
                             w[k] = pack_bf16(s[2 * k], s[2 * k + 1]);
-                            sum += bf16_lo(w[k]) + bf16_hi(w[k]);
+                            sum += bf16_lo(w[k]);
+                            sum2 += bf16_hi(w[k]);
                         }
                         tmem_st16u(pa, w);
                         tmem_st_wait();
-                        lq += sum;
+                        lq += sum + sum2;
                     }
                     if (ttok0 + PTOK > T) fence_proxy_async();
                     tc_fence_before();
