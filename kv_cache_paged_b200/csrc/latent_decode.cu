@@ -46,12 +46,12 @@ template <int DC, int TOK>
 struct LatCfg {
     static constexpr int KCH = (DC + 64) / 64;           // 64-wide K chunks: latent, then rope
     static constexpr int NVC = DC / DV;                   // value slices
-    static constexpr uint32_t Q_BYTES = KCH * 128 * 128;  // 128 rows x 128 B per chunk
+    static constexpr uint32_t Q_BYTES = 128 * 128;        // q's rope chunk: 128 rows x 128 B
     static constexpr uint32_t CHUNK = TOK * 128;          // one 64-dim chunk of a tile
     static constexpr uint32_t STAGE = KCH * CHUNK;
     static constexpr uint32_t S_COL = DV;                 // TMEM columns of the two S buffers
-    static constexpr uint32_t P_COL = DV + 2 * TOK;       // TMEM columns of the two P buffers
-    static constexpr uint32_t P_COLS = TOK / 2;           // bf16 pairs per row
+    static constexpr uint32_t Q_COL = DV + 2 * TOK;       // TMEM columns of q's latent part (bf16 pairs)
+    static_assert(DC == DV && Q_COL + DC / 2 <= 512, "q's latent part must fit in tensor memory");
 };
 
 template <int DC, int TOK>
@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(384, 1)
     using C = LatCfg<DC, TOK>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
-    __shared__ uint64_t qfull_bar, qempty_bar, sfull_bar[2], sfree_bar[2], pfull_bar[2], pfree_bar[2], end_bar;
+    __shared__ uint64_t qfull_bar, qtm_bar, qempty_bar, sfull_bar[2], pfull_bar[2], pfree_bar[2], end_bar;
     __shared__ Seg segs[LMAXSEG];
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
@@ -89,11 +89,11 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(&qfull_bar, 1);
+        mbar_init(&qfull_bar, 1);  // q's rope chunk (TMA)
+        mbar_init(&qtm_bar, 4);    // q's latent part written into tensor memory by softmax warps 4..7
         mbar_init(&qempty_bar, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sfull_bar[s], 1);
-            mbar_init(&sfree_bar[s], 8);
             mbar_init(&pfull_bar[s], 8);
             mbar_init(&pfree_bar[s], 1);
         }
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(384, 1)
     // counters that persist across segment-list rounds
     uint32_t p_issued = 0, p_qloads = 0;                    // producer
     uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;        // MMA issuer
-    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0;        // softmax
+    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0, x_q = 0;  // softmax
 
     for (int skip = 0;; skip += LMAXSEG) {
         if (warp == 0) {
@@ -147,13 +147,12 @@ __global__ void __launch_bounds__(384, 1)
                     break;
                 }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&qfull_bar, (uint32_t)rows_tile * C::KCH * 128);
+                    mbar_arrive_expect_tx(&qfull_bar, (uint32_t)rows_tile * 128);
                     for (int run = 0; run * rb < rows_tile; ++run) {
                         const int n0 = rt * 128 + run * rb;
                         const int i = n0 / g, h0 = n0 % g;
                         const int row = (sg.b * a.L + i) * a.h_q + c * g + h0;
-                        for (int ch = 0; ch < C::KCH; ++ch)
-                            tma_load_3d(q_s + ch * 16384 + run * rb * 128, &qmap, &qfull_bar, 0, row, ch, pol);
+                        tma_load_3d(q_s + run * rb * 128, &qmap, &qfull_bar, 0, row, C::KCH - 1, pol);
                     }
                 }
                 ++p_qloads;
@@ -209,18 +208,24 @@ __global__ void __launch_bounds__(384, 1)
                 auto issue_s = [&](uint32_t gt) -> bool {
                     const uint32_t stage = gt % nstage;
                     if (!mbar_wait_one(&full_bar[stage], (gt / nstage) & 1, &abort_sh, a.err, lim_ns)) return false;
+                    // S(j) goes into buffer j & 1, over P(j - 2): the MMAs of one thread run in
+                    // issue order, so this product, issued after the P.V product of tile j - 2,
+                    // cannot overwrite that P before it is read
                     const uint32_t sb = m_s & 1;
-                    if (!mbar_wait_one(&sfree_bar[sb], ((m_s >> 1) & 1) ^ 1, &abort_sh, a.err, lim_ns)) return false;
                     tc_fence_after();
                     const uint32_t d = tmem + C::S_COL + sb * TOK;
                     // descriptors advance by (byte offset >> 4) in their low word: one add per MMA
                     const uint64_t dk0 = umma_desc(st0 + stage * C::STAGE, 16, 1024, 2);
 #pragma unroll
-                    for (int kc = 0; kc < C::KCH; ++kc)
+                    for (int kc = 0; kc < C::KCH - 1; ++kc)  // latent chunks: q from tensor memory
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(d, dq0 + (uint64_t)((kc * 16384 + kk * 32) >> 4),
-                                      dk0 + (uint64_t)((kc * C::CHUNK + kk * 32) >> 4), idesc_s, (kc | kk) != 0);
+                            umma_bf16_ts(d, tmem + C::Q_COL + kc * 32 + kk * 8,
+                                         dk0 + (uint64_t)((kc * C::CHUNK + kk * 32) >> 4), idesc_s, (kc | kk) != 0);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // rope chunk: q from shared memory
+                        umma_bf16(d, dq0 + (uint64_t)((kk * 32) >> 4),
+                                  dk0 + (uint64_t)(((C::KCH - 1) * C::CHUNK + kk * 32) >> 4), idesc_s, 1u);
                     umma_commit(&sfull_bar[sb]);
                     ++m_s;
                     return true;
@@ -228,6 +233,7 @@ __global__ void __launch_bounds__(384, 1)
                 for (int si = 0; si < nseg && ok; ++si) {
                     const int n = segs[si].t1 - segs[si].t0;
                     if (!mbar_wait_one(&qfull_bar, m_q & 1, &abort_sh, a.err, lim_ns)) break;
+                    if (!mbar_wait_one(&qtm_bar, m_q & 1, &abort_sh, a.err, lim_ns)) break;
                     ++m_q;
                     tc_fence_after();
                     if (!issue_s(m_tile)) break;
@@ -248,7 +254,7 @@ __global__ void __launch_bounds__(384, 1)
                         tc_fence_after();
                         const uint32_t stage = (m_tile + j) % nstage;
                         const uint64_t dv0 = umma_desc(st0 + stage * C::STAGE + vc * 4 * C::CHUNK, C::CHUNK, 1024, 2);
-                        const uint32_t pa = tmem + C::P_COL + pb * C::P_COLS;
+                        const uint32_t pa = tmem + C::S_COL + pb * TOK;  // P(j) over S(j)
 #pragma unroll
                         for (int kk = 0; kk < TOK / 16; ++kk)
                             umma_bf16_ts(tmem, pa + kk * 8, dv0 + (uint64_t)(kk * 128), idesc_pv,
@@ -286,9 +292,11 @@ __global__ void __launch_bounds__(384, 1)
             auto exchange = [&](float v, float &other) -> bool {
                 const int buf = x_x & 1;
                 xchg_sh[buf][hf][r] = v;
+                tc_fence_before();  // this warp's tensor-memory reads happen before the arrival
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&xbar);
                 if (!mbar_wait_warp(&xbar, x_x & 1, &abort_sh, a.err, lim_ns)) return false;
+                tc_fence_after();
                 other = xchg_sh[buf][hf ^ 1][r];
                 ++x_x;
                 return true;
@@ -298,6 +306,35 @@ __global__ void __launch_bounds__(384, 1)
                 const int b = sg.b;
                 const int T = clamp_len(__ldg(a.seqlens + b), max_tokens, a.L, nullptr);
                 const int lim = row_ok ? T - a.L + i_row : -1;
+                if (hf == 0) {
+                    // q's latent part of this segment's rows -> tensor memory (the A operand of
+                    // the score product), once the previous segment's score MMAs are done with it
+                    if (!mbar_wait_warp(&qempty_bar, (x_q & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint4 *src =
+                        row_ok ? (const uint4 *)(a.q + ((size_t)(b * a.L + i_row) * a.h_q + head) * (DC + 64)) : nullptr;
+#pragma unroll 1
+                    for (int part16 = 0; part16 < DC / 32; ++part16) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint4 v = src ? __ldg(src + part16 * 4 + k) : make_uint4(0, 0, 0, 0);
+                            w[4 * k] = v.x;
+                            w[4 * k + 1] = v.y;
+                            w[4 * k + 2] = v.z;
+                            w[4 * k + 3] = v.w;
+                        }
+                        tmem_st16u(tmem + lane_base + C::Q_COL + part16 * 16, w);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&qtm_bar);
+                }
+                ++x_q;
                 // l: sum of the fp32 P (gives lse); lq: sum of the bf16-rounded P the product
                 // uses (normalises O: a convex combination of the rounded weights).  Both are
                 // partial over this thread's columns until the epilogue.
@@ -319,9 +356,6 @@ __global__ void __launch_bounds__(384, 1)
                             tmem_ld16(tmem + lane_base + C::S_COL + sb * TOK + hf * HC, s);
                         }
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sfree_bar[sb]);
                     ++x_s;
                     const bool full = tile * TOK + TOK - 1 <= T - a.L && row_ok;  // no column masked
                     if (warp_live) mx = tile_max(s, full, tok0, lim, a.scale_log2);
@@ -377,15 +411,10 @@ __global__ void __launch_bounds__(384, 1)
                             *(uint4 *)(v0 + ch * C::CHUNK + row * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                         }
                     }
-                    // P (bf16 pairs) -> tensor memory buffer x_pv & 1, once the P.V that last read
-                    // that buffer has completed
-                    if (x_pv >= 2 && !wait_pv(x_pv - 2)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+                    // P (bf16 pairs) over S in buffer x_pv & 1: both halves have read their S
+                    // columns (the row-max exchange above orders that)
                     if (warp_live) {
-                        const uint32_t pa = tmem + lane_base + C::P_COL + (x_pv & 1) * C::P_COLS + hf * (HC / 2);
+                        const uint32_t pa = tmem + lane_base + C::S_COL + sb * TOK + hf * (HC / 2);
                         uint32_t w[HC / 2];
                         float sum = 0.f, sum2 = 0.f;
 #pragma unroll
