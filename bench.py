@@ -39,7 +39,9 @@ UNIT = "us/step"
 FALLBACK_HBM_GBS, FALLBACK_TFLOPS = 6650.0, 1590.0
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 KERNEL_SOURCES = {"group": ["kv_cache_paged_b200/csrc/group_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"],
-                  "latent": ["kv_cache_paged_b200/csrc/latent_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"]}
+                  "latent": ["kv_cache_paged_b200/csrc/latent_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"],
+                  "pair": ["kv_cache_paged_b200/csrc/latent_pair.cu", "kv_cache_paged_b200/csrc/common.cuh"]}
+KERNEL_NAMES = {"group": "group_decode_kernel", "latent": "latent_decode_kernel", "pair": "mla_pair_kernel"}
 
 
 def describe(inp):
@@ -373,7 +375,7 @@ def main():
     t_step, t_kern, t_e2e = max_over_ranks([t_step, t_kern, t_e2e], pg, device=dev)
 
     hbm, tfl, peak_src = load_peaks()
-    variant_kind = "latent" if inp.variant == "gla" else "group"
+    variant_kind = ("pair" if inp.d == 512 else "latent") if inp.variant == "gla" else "group"
     tensor_bound = flops / (tfl * 1e12) > nbytes / (hbm * 1e9)
     if tensor_bound:
         achieved = flops / (t_kern * 1e-3) / 1e12
@@ -382,7 +384,7 @@ def main():
         achieved = nbytes / (t_kern * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm}
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
-    roof["kernel"] = "group_decode_kernel" if variant_kind == "group" else "latent_decode_kernel"
+    roof["kernel"] = KERNEL_NAMES[variant_kind]
     roof["kernel_us"] = t_kern * 1e3
     roof["traffic"] = committed_traffic(variant_kind, args.workload, inp.L)
     roof["roofline_us"] = accounting.roofline_us(nbytes, flops, hbm, tfl)
