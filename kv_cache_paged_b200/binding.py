@@ -1,4 +1,4 @@
-"""Thin ctypes binding over the C-ABI in include/kvdecode.h.
+"""Thin ctypes binding over the C-ABI in include/kvdecode.h and include/kvappend.h.
 
 Argument marshalling only: tensors are checked for dtype/shape/device and their
 device pointers, together with torch's current CUDA stream, are handed to the
@@ -14,7 +14,8 @@ import threading
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "_lib", "libkvdecode.so")
-HEADER = os.path.join(os.path.dirname(HERE), "include", "kvdecode.h")
+INCLUDE = os.path.join(os.path.dirname(HERE), "include")
+HEADER = os.path.join(INCLUDE, "kvdecode.h")
 
 KVD_OK = 0
 STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "workspace too small",
@@ -47,6 +48,27 @@ class GLAParams(ctypes.Structure):
                 ("B", _i32), ("L", _i32), ("h_q", _i32), ("h_c", _i32), ("d_c", _i32), ("d_r", _i32),
                 ("page_size", _i32), ("num_pages", _i32), ("max_pages", _i32), ("scale", ctypes.c_float),
                 ("num_parts", _i32)]
+
+
+class GQAAppendParams(ctypes.Structure):
+    _fields_ = [("k_new", _vp), ("v_new", _vp), ("k_cache", _vp), ("v_cache", _vp), ("positions", _vp),
+                ("slot_mapping", _vp), ("error_word", _vp),
+                ("N", _i32), ("h_kv", _i32), ("d", _i32), ("d_r", _i32), ("num_rows", _i32),
+                ("rope_base", ctypes.c_float)]
+
+
+class GTAAppendParams(ctypes.Structure):
+    _fields_ = [("tied_new", _vp), ("rope_new", _vp), ("tied_cache", _vp), ("rope_cache", _vp), ("positions", _vp),
+                ("slot_mapping", _vp), ("error_word", _vp),
+                ("N", _i32), ("h_kv", _i32), ("d_h", _i32), ("d_r", _i32), ("num_rows", _i32),
+                ("rope_base", ctypes.c_float)]
+
+
+class GLAAppendParams(ctypes.Structure):
+    _fields_ = [("latent_new", _vp), ("rope_new", _vp), ("latent_cache", _vp), ("rope_cache", _vp),
+                ("positions", _vp), ("slot_mapping", _vp), ("error_word", _vp),
+                ("N", _i32), ("h_c", _i32), ("d_c", _i32), ("d_r", _i32), ("num_rows", _i32),
+                ("rope_base", ctypes.c_float)]
 
 
 _lib = None
@@ -89,15 +111,24 @@ def lib():
             L.kvd_status_string.restype = ctypes.c_char_p
             L.kvd_status_string.argtypes = [ctypes.c_int]
             L.kvd_version.restype = ctypes.c_int
+            for name, P in (("gqa", GQAAppendParams), ("gta", GTAAppendParams), ("gla", GLAAppendParams)):
+                f = getattr(L, f"kvd_{name}_append")
+                f.restype = ctypes.c_int
+                f.argtypes = [ctypes.POINTER(P), _vp]
+            L.kvd_rope_q.restype = ctypes.c_int
+            L.kvd_rope_q.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_float, _vp]
             _lib = L
     return _lib
 
 
 def header_functions():
-    """Names of the functions include/kvdecode.h declares."""
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(kvd_[a-z0-9_]+)\s*\(", text)))
+    """Names of the functions the headers under include/ declare."""
+    names = set()
+    for h in sorted(os.listdir(INCLUDE)):
+        if h.endswith(".h"):
+            text = re.sub(r"/\*.*?\*/", "", open(os.path.join(INCLUDE, h)).read(), flags=re.S)
+            names.update(re.findall(r"\b(kvd_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def _check(fn, status):
@@ -272,3 +303,70 @@ def num_sms():
     if n < 0:
         raise KVDecodeError("kvd_num_sms", n)
     return n
+
+
+# ----------------------------------------------------------------------------- cache append + RoPE
+def _append_common(positions, slot_mapping, N, error_word):
+    torch = _torch()
+    pos = _dev(positions, "positions", torch.int32, 1)
+    slot = _dev(slot_mapping, "slot_mapping", torch.int32, 1)
+    if positions.shape[0] != N or slot_mapping.shape[0] != N:
+        raise ValueError("positions and slot_mapping need one entry per new token")
+    err = _dev(error_word, "error_word", torch.int32) if error_word is not None else None
+    return pos, slot, err
+
+
+def _rows(cache, name):
+    return cache.shape[0] * cache.shape[1]
+
+
+def gqa_append(k_new, v_new, positions, slot_mapping, k_cache, v_cache, d_r, *, rope_base=10000.0,
+               error_word=None, stream=None):
+    """Write N new tokens: k_new/v_new [N, h_kv, d] -> caches [P, S, h_kv, d] at slot_mapping rows,
+    RoPE on the last d_r dims of each K head at `positions`."""
+    torch = _torch()
+    N, h_kv, d = k_new.shape
+    pos, slot, err = _append_common(positions, slot_mapping, N, error_word)
+    p = GQAAppendParams(_dev(k_new, "k_new", torch.bfloat16, 3), _dev(v_new, "v_new", torch.bfloat16, 3),
+                        _dev(k_cache, "k_cache", torch.bfloat16, 4), _dev(v_cache, "v_cache", torch.bfloat16, 4),
+                        pos, slot, err, N, h_kv, d, d_r, _rows(k_cache, "k_cache"), rope_base)
+    _check("kvd_gqa_append", lib().kvd_gqa_append(ctypes.byref(p), _stream_ptr(stream)))
+
+
+def gta_append(tied_new, rope_new, positions, slot_mapping, tied_cache, rope_cache, *, rope_base=10000.0,
+               error_word=None, stream=None):
+    """Write N new tokens: tied_new [N, h_kv, d_h] as is, rope_new [N, d_r] rotated to `positions`."""
+    torch = _torch()
+    N, h_kv, d_h = tied_new.shape
+    d_r = rope_new.shape[1]
+    pos, slot, err = _append_common(positions, slot_mapping, N, error_word)
+    p = GTAAppendParams(_dev(tied_new, "tied_new", torch.bfloat16, 3), _dev(rope_new, "rope_new", torch.bfloat16, 2),
+                        _dev(tied_cache, "tied_cache", torch.bfloat16, 4),
+                        _dev(rope_cache, "rope_cache", torch.bfloat16, 3),
+                        pos, slot, err, N, h_kv, d_h, d_r, _rows(tied_cache, "tied_cache"), rope_base)
+    _check("kvd_gta_append", lib().kvd_gta_append(ctypes.byref(p), _stream_ptr(stream)))
+
+
+def gla_append(latent_new, rope_new, positions, slot_mapping, latent_cache, rope_cache, *, rope_base=10000.0,
+               error_word=None, stream=None):
+    """Write N new tokens: latent_new [N, h_c, d_c] as is, rope_new [N, d_r] rotated to `positions`."""
+    torch = _torch()
+    N, h_c, d_c = latent_new.shape
+    d_r = rope_new.shape[1]
+    pos, slot, err = _append_common(positions, slot_mapping, N, error_word)
+    p = GLAAppendParams(_dev(latent_new, "latent_new", torch.bfloat16, 3),
+                        _dev(rope_new, "rope_new", torch.bfloat16, 2),
+                        _dev(latent_cache, "latent_cache", torch.bfloat16, 4),
+                        _dev(rope_cache, "rope_cache", torch.bfloat16, 3),
+                        pos, slot, err, N, h_c, d_c, d_r, _rows(latent_cache, "latent_cache"), rope_base)
+    _check("kvd_gla_append", lib().kvd_gla_append(ctypes.byref(p), _stream_ptr(stream)))
+
+
+def rope_q(q, seqlens, rope_off, d_r, *, rope_base=10000.0, stream=None):
+    """Rotate q [B, L, heads, d_qk] in place: dims [rope_off, rope_off + d_r) of row (b, i) go to
+    position seqlens[b] - L + i."""
+    torch = _torch()
+    B, L, heads, d_qk = q.shape
+    st = lib().kvd_rope_q(_dev(q, "q", torch.bfloat16, 4), _dev(seqlens, "seqlens", torch.int32, 1), B, L, heads,
+                          d_qk, rope_off, d_r, rope_base, _stream_ptr(stream))
+    _check("kvd_rope_q", st)
