@@ -221,6 +221,153 @@ def run_reference(args, inp, cfg, rank):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- cache append
+APPEND_SHAPES = {  # per token: (plain heads, plain dim, rope slices, d_r, rope inside the key heads)
+    "append_gta": dict(kind="gta", heads=8, dim=128, d_r=64),
+    "append_gqa": dict(kind="gqa", heads=8, dim=128, d_r=128),
+    "append_mla": dict(kind="gla", heads=1, dim=512, d_r=64),
+    "append_gla2": dict(kind="gla", heads=2, dim=256, d_r=64),
+}
+APPEND_METRIC = "cache append (state copy + RoPE) us/call and GB/s as % of B200 HBM peak (1 GPU)"
+
+
+def append_bytes(sh, n):
+    """Algorithmic bytes of one append of n tokens: every stored element read once and written once,
+    plus the positions and slot indices."""
+    if sh["kind"] == "gqa":
+        elems = 2 * sh["heads"] * sh["dim"]
+    else:
+        elems = sh["heads"] * sh["dim"] + sh["d_r"]
+    return n * (elems * 2 * 2 + 8)
+
+
+def append_inputs(sh, n, seed=31):
+    rng = np.random.default_rng(seed)
+    rows = ((n + 63) // 64 + 8) * 64
+    f = lambda shape: wl.f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32))
+    if sh["kind"] == "gqa":
+        srcs = [f((n, sh["heads"], sh["dim"])), f((n, sh["heads"], sh["dim"]))]
+        dsts = [(rows // 64, 64, sh["heads"], sh["dim"])] * 2
+    else:
+        srcs = [f((n, sh["heads"], sh["dim"])), f((n, sh["d_r"]))]
+        dsts = [(rows // 64, 64, sh["heads"], sh["dim"]), (rows // 64, 64, sh["d_r"])]
+    pos = rng.integers(0, 65536, n).astype(np.int32)
+    slot = rng.permutation(rows)[:n].astype(np.int32)
+    return srcs, dsts, pos, slot
+
+
+def oracle_append(sh, srcs, pos, n):
+    """The reference arm for the append: the oracle's fp64 rotation of every RoPE slice plus a copy."""
+    from oracle import oracle as orc
+    x = wl.bf16_bits_to_f32(srcs[0][:n] if sh["kind"] == "gqa" else srcs[1][:n]).astype(np.float64)
+    for t in range(n):
+        if sh["kind"] == "gqa":
+            for h in range(sh["heads"]):
+                orc.rope(x[t, h, sh["dim"] - sh["d_r"]:], float(pos[t]))
+        else:
+            orc.rope(x[t], float(pos[t]))
+    return [np.copy(a[:n]) for a in srcs]
+
+
+def run_append(args, rank):
+    sh = APPEND_SHAPES[args.workload]
+    n = args.tokens
+    nbytes = append_bytes(sh, n)
+    cfg = {"workload": f"{sh['kind'].upper()} cache append of {n} tokens into a paged cache (page 64, random "
+                       f"slot_mapping, positions in [0, 65536)), heads {sh['heads']} x {sh['dim']}, d_r {sh['d_r']}",
+           "tokens": n, "algorithmic_bytes_per_call": int(nbytes), "parallelism": "replicas1",
+           "l2": "a 256 MiB read evicts L2 before every timed call"}
+    srcs, dsts, pos, slot = append_inputs(sh, n)
+    # the oracle on a bounded sample, scaled to the call (rank 0, N = 1 only)
+    t_cpu = None
+    if rank == 0 and (args.impl == "reference" or not args.no_cpu_baseline):
+        m = min(n, 2048)
+        t0 = time.perf_counter()
+        oracle_append(sh, srcs, pos, m)
+        t_cpu = (time.perf_counter() - t0) / m * n * 1e6
+        cpu = {"value": t_cpu, "unit": "us/call", "cores": 1, "kind": "oracle",
+               "sample": f"{m} of {n} tokens, time scaled to the call"}
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps({"impl": "reference", "metric": APPEND_METRIC, "value": t_cpu, "unit": "us/call",
+                              "n_gpus": args.gpus, "steps": 1, "warmup": 0, "ms_per_step": t_cpu / 1e3,
+                              "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                              "data": "synthetic", "config": cfg, "cpu_baseline": cpu,
+                              "e2e": {"value": t_cpu, "unit": "us/call", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}), flush=True)
+        return
+    import torch
+    from kv_cache_paged_b200 import binding
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    s0, s1 = bf(srcs[0]), bf(srcs[1])
+    c0 = torch.zeros(dsts[0], dtype=torch.bfloat16, device=dev)
+    c1 = torch.zeros(dsts[1], dtype=torch.bfloat16, device=dev)
+    dpos, dslot = torch.from_numpy(pos).to(dev), torch.from_numpy(slot).to(dev)
+    flush = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    st = torch.cuda.Stream(device=dev)
+
+    def call():
+        if sh["kind"] == "gqa":
+            binding.gqa_append(s0, s1, dpos, dslot, c0, c1, sh["d_r"], stream=st)
+        elif sh["kind"] == "gta":
+            binding.gta_append(s0, s1, dpos, dslot, c0, c1, stream=st)
+        else:
+            binding.gla_append(s0, s1, dpos, dslot, c0, c1, stream=st)
+
+    with torch.cuda.stream(st):
+        for _ in range(args.warmup):
+            flush.max()
+            call()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        clk = ClockSampler(dev.index)
+        clk.start()
+        clk.mark_on()
+        for a, b in ev:
+            flush.max()
+            a.record(st)
+            call()
+            b.record(st)
+        torch.cuda.synchronize()
+        clk.mark_off()
+        clocks = clk.stop()
+        us = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+        # end to end: the new tokens' inputs from pinned host memory, the call, one word back
+        hs = [torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).pin_memory() for x in srcs]
+        hp, hsl = torch.from_numpy(pos).pin_memory(), torch.from_numpy(slot).pin_memory()
+        e2e = []
+        for _ in range(max(3, args.steps // 4)):
+            flush.max()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            s0.view(torch.int16).copy_(hs[0], non_blocking=True)
+            s1.view(torch.int16).copy_(hs[1], non_blocking=True)
+            dpos.copy_(hp, non_blocking=True)
+            dslot.copy_(hsl, non_blocking=True)
+            call()
+            word = c1.view(-1)[:1].cpu()
+            b.record(st)
+            torch.cuda.synchronize()
+            e2e.append(a.elapsed_time(b) * 1e3)
+    hbm, _, src = load_peaks()
+    ach = nbytes / (us * 1e-6) / 1e9
+    h2d = sum(x.nbytes for x in srcs) + pos.nbytes + slot.nbytes
+    line = {"metric": APPEND_METRIC, "value": us, "unit": "us/call", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 copy, f64 rotation", "data": "synthetic", "config": cfg,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                         "traffic": None, "peak_source": src, "kernel": "append_kernel", "kernel_us": us},
+            "e2e": {"value": statistics.mean(e2e), "unit": "us/call", "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": 2},
+            "gpu_launches": args.steps, "clocks": clocks}
+    if t_cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -228,7 +375,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="kvd", choices=["kvd", "reference"])
-    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny"])
+    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny"] + list(APPEND_SHAPES))
+    ap.add_argument("--tokens", type=int, default=65536, help="new tokens per call (append workloads)")
     ap.add_argument("--qlen", type=int, default=1)
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -240,6 +388,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", 1))
     local = int(os.environ.get("LOCAL_RANK", 0))
 
+    if args.workload in APPEND_SHAPES:
+        run_append(args, rank)
+        return
     inp = wl.make_workload(args.workload, L=args.qlen)
     nbytes, flops, kvb = accounting.of_inputs(inp)
     cfg = {"workload": describe(inp), "global_batch": inp.B * world, "seq_len": int(inp.seqlens.max()),
