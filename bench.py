@@ -378,6 +378,7 @@ def main():
     ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny"] + list(APPEND_SHAPES))
     ap.add_argument("--tokens", type=int, default=65536, help="new tokens per call (append workloads)")
     ap.add_argument("--qlen", type=int, default=1)
+    ap.add_argument("--page-size", type=int, default=0, help="override the workload's page size (tokens per page)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
@@ -391,7 +392,8 @@ def main():
     if args.workload in APPEND_SHAPES:
         run_append(args, rank)
         return
-    inp = wl.make_workload(args.workload, L=args.qlen)
+    over = {"page_size": args.page_size} if args.page_size > 0 else {}
+    inp = wl.make_workload(args.workload, L=args.qlen, **over)
     nbytes, flops, kvb = accounting.of_inputs(inp)
     cfg = {"workload": describe(inp), "global_batch": inp.B * world, "seq_len": int(inp.seqlens.max()),
            "q_len": inp.L, "seed": wl.SEEDS[args.workload], "parallelism": f"replicas{world}",

@@ -72,6 +72,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // ----------------------------------------------------------------------------- GQA / GTA
 struct GroupPlan {
     int gpc, n_sub, parts, nt, nstage, tile;
+    bool gather;
     uint32_t stage_bytes, stage_bytes_tx;
     size_t ws_bytes;
 };
@@ -92,7 +93,6 @@ int plan_group(bool tied, const void *q, const void *c0, const void *c1, const i
     if (tied) {
         if ((d_r != 32 && d_r != 64) || d_r > d || (d - d_r) % 16) return KVD_ERR_UNSUPPORTED_SHAPE;
     }
-    if (S % TILE) return KVD_ERR_UNSUPPORTED_SHAPE;
     if ((long long)P * S >= (1ll << 31) || (long long)max_pages * S >= (1ll << 31)) return KVD_ERR_UNSUPPORTED_SHAPE;
     const int R = (h_q / h_kv) * L;
     int nt = R <= 8 ? 1 : R <= 16 ? 2 : R <= 32 ? 4 : 0;
@@ -109,8 +109,17 @@ int plan_group(bool tied, const void *q, const void *c0, const void *c1, const i
         const uint32_t kvt = (uint32_t)gpc * d * tt * 2;
         return tied ? kvt + tt * d_r * 2 : 2 * kvt;
     };
+    // Pages that hold whole tiles are loaded with one box per operand; smaller (or ragged)
+    // pages are gathered row by row (four rows per TMA).
+    const bool fits32 = nt == 1 && 3 * round_up(stage_tx(32), 1024) <= SMEM_BUDGET - 1024;
     int tile = TILE;
-    if (nt == 1 && S % 32 == 0 && 3 * round_up(stage_tx(32), 1024) <= SMEM_BUDGET - 1024) tile = 32;
+    bool gather = false;
+    if (S % 32 == 0 && fits32) {
+        tile = 32;
+    } else if (S % TILE) {
+        gather = true;
+        tile = fits32 ? 32 : TILE;
+    }
     const uint32_t tx = stage_tx(tile);
     const uint32_t stage = (uint32_t)round_up(tx, 1024);
     int nstage = (int)((SMEM_BUDGET - 1024) / stage);
@@ -131,6 +140,7 @@ int plan_group(bool tied, const void *q, const void *c0, const void *c1, const i
     gp->nt = nt;
     gp->nstage = nstage;
     gp->tile = tile;
+    gp->gather = gather;
     gp->stage_bytes = stage;
     gp->stage_bytes_tx = tx;
     gp->ws_bytes = WS_HEADER + round_up(slots * rows * 4, 256) + slots * rows * d * 4;
@@ -150,20 +160,23 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
 
     CUtensorMap m0, m1;
     const cuuint64_t tokens = (cuuint64_t)P * S;
-    {
+    if (gp.gather) {
+        memset(&m0, 0, sizeof(m0));  // rows are copied with cp.async; no tensor maps
+        memset(&m1, 0, sizeof(m1));
+    } else {
         cuuint64_t dims[3] = {64, tokens, (cuuint64_t)h_kv * d / 64};
         cuuint64_t strides[2] = {(cuuint64_t)h_kv * d * 2, 128};
         cuuint32_t box[3] = {64, (cuuint32_t)gp.tile, (cuuint32_t)(gp.gpc * d / 64)};
         if (!encode(&m0, c0, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
         if (!tied && !encode(&m1, c1, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
-    }
-    if (tied) {
-        cuuint64_t dims[2] = {(cuuint64_t)d_r, tokens};
-        cuuint64_t strides[1] = {(cuuint64_t)d_r * 2};
-        cuuint32_t box[2] = {(cuuint32_t)d_r, (cuuint32_t)gp.tile};
-        if (!encode(&m1, c1, 2, dims, strides, box,
-                    d_r == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
-            return KVD_ERR_CUDA;
+        if (tied) {
+            cuuint64_t rdims[2] = {(cuuint64_t)d_r, tokens};
+            cuuint64_t rstrides[1] = {(cuuint64_t)d_r * 2};
+            cuuint32_t rbox[2] = {(cuuint32_t)d_r, (cuuint32_t)gp.tile};
+            if (!encode(&m1, c1, 2, rdims, rstrides, rbox,
+                        d_r == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+                return KVD_ERR_CUDA;
+        }
     }
 
     const size_t slots = (size_t)B + gp.parts - 1;
@@ -186,6 +199,9 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
     a.num_pages = P;
     a.max_pages = max_pages;
     a.tile = gp.tile;
+    a.gather = gp.gather ? 1 : 0;
+    a.cache0 = c0;
+    a.cache1 = c1;
     a.gpc = gp.gpc;
     a.n_sub = gp.n_sub;
     a.parts = gp.parts;

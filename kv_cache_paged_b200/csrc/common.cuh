@@ -203,6 +203,16 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
         "l"(m), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
         : "memory");
 }
+// 16-byte copy global -> shared through L2 only (cp.async.cg), with an L2 cache policy.
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src, uint64_t policy) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "l"(policy)
+                 : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed (no count increment:
+// the barrier's expected count must include this arrival).
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 // L2 policy for data read exactly once (the KV stream).
 __device__ __forceinline__ uint64_t policy_evict_first() {
     uint64_t p;

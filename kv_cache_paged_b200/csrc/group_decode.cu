@@ -29,9 +29,10 @@ namespace kvd {
 namespace {
 
 constexpr int MAXSEG = 128;
+constexpr int GATHER_WARPS = 4;  // producer warps when tiles are gathered token by token
 
 template <bool TIED, int D, int DR, int NT, int TT>
-__global__ void __launch_bounds__(9 * 32, 1)
+__global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
     group_decode_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
                         const GroupArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -53,13 +54,13 @@ __global__ void __launch_bounds__(9 * 32, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nstage; ++s) {
-            mbar_init(&full_bar[s], 1);
+            mbar_init(&full_bar[s], a.gather ? 32 * GATHER_WARPS : 1);  // gathered: every producer lane
             mbar_init(&empty_bar[s], gpc);
         }
         abort_sh = 0;
         fence_mbar_init();
     }
-    if (warp == gpc && lane == 0) {
+    if (warp == gpc && lane == 0 && !a.gather) {
         tma_prefetch_desc(&map0);
         tma_prefetch_desc(&map1);
     }
@@ -82,8 +83,8 @@ __global__ void __launch_bounds__(9 * 32, 1)
         __syncthreads();
         const int nseg = nseg_sh;
 
-        if (warp == gpc) {
-            // ------------------------------------------------------------ producer
+        if (warp >= gpc) {
+            // ------------------------------------------------------------ producer(s)
             const uint64_t pol = policy_evict_first();
             const int z0 = sub * gpc * (D / 64);  // first 64-wide chunk of this CTA's groups
             uint32_t issued = it;
@@ -91,6 +92,68 @@ __global__ void __launch_bounds__(9 * 32, 1)
             for (int si = 0; si < nseg && !stop; ++si) {
                 const Seg sg = segs[si];
                 const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
+                if (a.gather) {
+                    // Pages smaller than a tile (down to one token) or not a multiple of it.  The
+                    // GATHER_WARPS producer warps all walk every tile; warp w copies the tokens
+                    // k = w, w + GATHER_WARPS, ...: one lane per token resolves its cache row
+                    // (distributed offset calculation, fetched a tile ahead), then the warp copies
+                    // each token's row with 16-byte cp.async into the same swizzled layout the box
+                    // loads produce (a token's row is contiguous: 32 lanes move 512 consecutive
+                    // bytes per instruction).  Every lane arrives on the stage's barrier when its
+                    // copies have landed.
+                    const int pw = warp - gpc;
+                    constexpr int TPW = TT / GATHER_WARPS;      // tokens per warp and tile
+                    const int T = clamp_len(__ldg(a.seqlens + sg.b), max_tokens, a.L, nullptr);
+                    const int nch = gpc * (D / 64);
+                    const size_t row_elems = (size_t)a.h_kv * D;
+                    const __nv_bfloat16 *c0 = (const __nv_bfloat16 *)a.cache0 + (size_t)z0 * 64;
+                    const __nv_bfloat16 *c1 = (const __nv_bfloat16 *)a.cache1 + (TIED ? 0 : (size_t)z0 * 64);
+                    constexpr int RU = TIED ? DR * 2 / 16 : 0;  // 16-byte units of a rope row
+                    // token of this lane in tile t (tokens past T_b repeat the last one; masked later)
+                    auto tok_of = [&](int t) { return min(t * TT + pw + GATHER_WARPS * lane, T - 1); };
+                    int nxt_tok = tok_of(sg.t0);
+                    int nxt_page = lane < TPW ? __ldg(bt + nxt_tok / a.page_size) : 0;
+                    for (int t = sg.t0; t < sg.t1 && !stop; ++t, ++issued) {
+                        const int tok = nxt_tok;
+                        int page = nxt_page;
+                        if (t + 1 < sg.t1) {
+                            nxt_tok = tok_of(t + 1);
+                            if (lane < TPW) nxt_page = __ldg(bt + nxt_tok / a.page_size);
+                        }
+                        const uint32_t stage = issued % nstage;
+                        if (!mbar_wait_warp(&empty_bar[stage], ((issued / nstage) & 1) ^ 1, &abort_sh, a.err,
+                                            a.wait_limit_ns)) {
+                            stop = true;
+                            break;
+                        }
+                        if (lane < TPW && (page < 0 || page >= a.num_pages)) {
+                            set_error(a.err, DEVERR_BAD_PAGE);
+                            page = 0;
+                        }
+                        const int myrow = page * a.page_size + tok % a.page_size;
+                        if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || issued != 0) {
+                            const uint32_t st = smem_u32(smem + (size_t)stage * a.stage_bytes);
+                            const int per_tok = nch * 8;  // 16-byte units of a token in K / tied / V
+#pragma unroll 1
+                            for (int i = 0; i < TPW; ++i) {
+                                const int k = pw + GATHER_WARPS * i;
+                                const int row = __shfl_sync(0xffffffffu, myrow, i);
+                                for (int u = lane; u < per_tok; u += 32) {
+                                    const int z = u >> 3, c = u & 7;
+                                    const uint32_t so = sw128((uint32_t)(z * TT + k), (uint32_t)c);
+                                    cp_async16(st + so, c0 + (size_t)row * row_elems + u * 8, pol);
+                                    if (!TIED) cp_async16(st + kv_tile + so, c1 + (size_t)row * row_elems + u * 8, pol);
+                                }
+                                if (TIED && lane < RU)
+                                    cp_async16(st + kv_tile + (DR == 64 ? sw128(k, lane) : sw64(k, lane)),
+                                               c1 + (size_t)row * DR + lane * 8, pol);
+                            }
+                            cp_async_arrive(&full_bar[stage]);
+                        }
+                    }
+                    continue;
+                }
+                if (warp != gpc) continue;  // whole-tile boxes: one producer warp
                 const int tiles_per_page = a.page_size / TT;
                 const int p_first = sg.t0 / tiles_per_page;
                 const int p_last = (sg.t1 - 1) / tiles_per_page;
@@ -130,7 +193,9 @@ __global__ void __launch_bounds__(9 * 32, 1)
                     }
                 }
             }
-            if (stop) {
+            if (stop && a.gather) {
+                asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's copies have landed
+            } else if (stop) {
                 // Let every copy already issued land before the CTA can exit.
                 const uint32_t lo = issued > (uint32_t)nstage ? issued - nstage : 0;
                 for (uint32_t k = lo; k < issued; ++k) {
@@ -415,7 +480,7 @@ cudaError_t launch_t(const CUtensorMap &m0, const CUtensorMap &m1, const GroupAr
     auto k = group_decode_kernel<TIED, D, DR, NT, TT>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, (a.gpc + 1) * 32, smem, st>>>(m0, m1, a);
+    k<<<grid, (a.gpc + (a.gather ? GATHER_WARPS : 1)) * 32, smem, st>>>(m0, m1, a);
     return cudaGetLastError();
 }
 

@@ -25,6 +25,8 @@ struct GroupArgs {
     uint32_t *err;
     int B, L, h_q, h_kv, page_size, num_pages, max_pages;
     int tile;   // tokens per pipeline stage (16 or 32)
+    int gather; // pages hold fewer tokens than a tile (or not a multiple): rows copied token by token
+    const void *cache0, *cache1;  // K / tied and V / rope caches (the gathered path reads them directly)
     int gpc;    // KV groups per CTA (consumer warps)
     int n_sub;  // CTAs per part = h_kv / gpc
     int parts;

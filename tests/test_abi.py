@@ -41,7 +41,6 @@ def _gta_params(**kw):
     (dict(L=0), -1),
     (dict(d_h=96), -2),                 # head dim outside the compiled set
     (dict(d_r=48), -2),
-    (dict(page_size=24), -2),           # not a multiple of the 16-token tile
     (dict(h_q=128, h_kv=2, L=1), -2),   # 64 rows per group: beyond the warp-MMA kernel
     (dict(scale=float("nan")), -1),
 ])
@@ -49,6 +48,12 @@ def test_gta_validation_errors(lib, kw, expect):
     p = _gta_params(**kw)
     assert lib.kvd_gta_workspace_size(ctypes.byref(p)) == 0
     assert lib.kvd_gta_decode(ctypes.byref(p), ctypes.c_void_p(256), 1 << 30, None) == expect
+
+
+@pytest.mark.parametrize("S", [1, 3, 24, 100])
+def test_any_page_size_is_accepted(lib, S):
+    """Pages that do not hold whole 16-token tiles are gathered row by row, not rejected."""
+    assert lib.kvd_gta_workspace_size(ctypes.byref(_gta_params(page_size=S))) > 0
 
 
 def test_workspace_size_and_too_small(lib):
