@@ -241,6 +241,7 @@ constexpr size_t SMEM_PER_BLOCK = 232448;
 constexpr size_t LATENT_STATIC_SMEM = 4096;
 
 struct LatentPlan {
+    bool spread;
     LatentShape shape;
     bool pair;
     int n_rt, n_vc, n_sub, parts, nstage, rb;
@@ -273,7 +274,10 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
     lp->n_vc = lp->pair ? 1 : p->d_c / 256;
     lp->n_sub = p->h_c * lp->n_rt * lp->n_vc;
     const int ctas_per_sub = lp->pair ? 2 : 1;
-    lp->rb = g < 128 ? g : 128;
+    // the GLA kernel spreads at most 64 rows over the four TMEM lane quadrants (16 each), which
+    // needs the q rows in 16-row runs that stay inside one query position
+    lp->spread = !lp->pair && R <= 64 && g % 16 == 0;
+    lp->rb = lp->spread ? 16 : (g < 128 ? g : 128);
     const size_t fixed = SMEM_PER_BLOCK - LATENT_STATIC_SMEM - 1024 - sh.q_bytes - sh.p_bytes;
     int nstage = (int)(fixed / sh.stage_bytes);
     if (nstage > MAX_STAGES) nstage = MAX_STAGES;
@@ -344,6 +348,7 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     a.max_pages = p->max_pages;
     a.n_sub = lp.n_sub;
     a.n_rt = lp.n_rt;
+    a.row_spread = lp.spread ? 1 : 0;
     a.parts = lp.parts;
     a.nstage = lp.nstage;
     a.scale_log2 = p->scale * 1.4426950408889634f;

@@ -53,6 +53,7 @@ struct LatentArgs {
     int B, L, h_q, h_c, page_size, num_pages, max_pages;
     int n_sub;  // CTAs per part = h_c * row blocks * value slices
     int n_rt;   // 128-row blocks per latent head
+    int row_spread;  // <= 64 rows, spread over lanes 0..15 of each TMEM lane quadrant (GLA kernel)
     int parts;
     int nstage;
     float scale_log2;

@@ -40,6 +40,8 @@ namespace {
 
 constexpr int LMAXSEG = 32;
 constexpr int DV = 256;  // value columns per CTA (fp32 accumulator columns in TMEM)
+constexpr int NSMX = 4;  // softmax warps, one per TMEM lane quadrant
+constexpr int LTHREADS = 32 * (4 + NSMX);  // warp 0 producer, 1 MMA, 2-3 idle, 4.. softmax
 constexpr float RESCALE_LOG2 = 8.f;
 
 template <int DC, int TOK>
@@ -55,7 +57,7 @@ struct LatCfg {
 };
 
 template <int DC, int TOK>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(LTHREADS, 1)
     latent_decode_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap latmap,
                          const __grid_constant__ CUtensorMap ropemap, const LatentArgs a) {
     using C = LatCfg<DC, TOK>;
@@ -66,8 +68,6 @@ __global__ void __launch_bounds__(384, 1)
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
     __shared__ uint32_t tmem_sh;
-    __shared__ uint64_t xbar;                 // row-value exchange between the two column halves
-    __shared__ float xchg_sh[2][2][128];
 
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *q_s = smem;
@@ -94,11 +94,10 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(&qempty_bar, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sfull_bar[s], 1);
-            mbar_init(&pfull_bar[s], 8);
+            mbar_init(&pfull_bar[s], NSMX);  // one arrival per softmax warp
             mbar_init(&pfree_bar[s], 1);
         }
         mbar_init(&end_bar, 1);
-        mbar_init(&xbar, 8);
         abort_sh = 0;
         fence_mbar_init();
     }
@@ -138,7 +137,7 @@ __global__ void __launch_bounds__(384, 1)
             // ================================================================ producer
             const uint64_t pol = policy_evict_first();
             bool stop = false;
-            const int rb = g < 128 ? g : 128;                      // q rows per TMA box
+            const int rb = a.row_spread ? 16 : (g < 128 ? g : 128);  // q rows per TMA box
             const int rows_tile = min(R - rt * 128, 128);          // valid rows of this row block
             for (int si = 0; si < nseg && !stop; ++si) {
                 const Seg sg = segs[si];
@@ -152,7 +151,9 @@ __global__ void __launch_bounds__(384, 1)
                         const int n0 = rt * 128 + run * rb;
                         const int i = n0 / g, h0 = n0 % g;
                         const int row = (sg.b * a.L + i) * a.h_q + c * g + h0;
-                        tma_load_3d(q_s + run * rb * 128, &qmap, &qfull_bar, 0, row, C::KCH - 1, pol);
+                        // spread rows: run k (rows 16k ..) lands at lanes 32k .. (see the softmax)
+                        const int srow = a.row_spread ? run * 32 : run * rb;
+                        tma_load_3d(q_s + srow * 128, &qmap, &qfull_bar, 0, row, C::KCH - 1, pol);
                     }
                 }
                 ++p_qloads;
@@ -269,18 +270,18 @@ __global__ void __launch_bounds__(384, 1)
             __syncwarp();
         } else if (warp >= 4) {
             // ================================================================ softmax / epilogue
-            // Eight warps: warp w reads TMEM lanes 32 (w % 4) .. + 31 (its rows) and the column
-            // half hf = (w - 4) / 4 of every S tile, of P and of O.  The two threads of a row
-            // exchange their tile maxima through shared memory so that they keep the same
-            // reference maximum; their partial sums are merged in the epilogue.
-            constexpr int HC = TOK / 2;                  // S / P columns per thread
-            const int st_id = threadIdx.x - 128;         // 0..255
-            const int hf = (warp - 4) >> 2;
-            const int r = (warp & 3) * 32 + lane;        // row = TMEM lane
+            // Four warps, one thread per row: warp w reads TMEM lanes 32 (w % 4) .. + 31 and the
+            // whole 64-token S row of its thread, so no row value crosses threads.  When a CTA has
+            // at most 64 rows (GLA-2 at q_len 1) they are spread over lanes 0..15 of every lane
+            // quadrant (row n at lane 32 (n / 16) + n % 16): each of the four warps, one per SM
+            // sub-partition, then holds 16 rows.
+            const int st_id = threadIdx.x - 128;         // 0 .. 127
+            const int r = (warp & 3) * 32 + lane;        // TMEM lane
             const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-            const int n_row = rt * 128 + r;
+            const bool spread = a.row_spread != 0;
+            const int n_row = spread ? ((lane < 16) ? (warp & 3) * 16 + lane : R) : rt * 128 + r;
             const bool row_ok = n_row < R;
-            const bool warp_live = rt * 128 + (warp & 3) * 32 < R;  // some row of this warp is real
+            const bool warp_live = spread || rt * 128 + (warp & 3) * 32 < R;  // some row of this warp is real
             const int i_row = row_ok ? n_row / g : 0;
             const int head = row_ok ? c * g + n_row % g : 0;
             bool ok = true;
@@ -288,25 +289,12 @@ __global__ void __launch_bounds__(384, 1)
             auto wait_pv = [&](uint32_t k) -> bool {
                 return mbar_wait_warp(&pfree_bar[k & 1], (k >> 1) & 1, &abort_sh, a.err, lim_ns);
             };
-            // exchange one float per row with the other column half (bounded barrier over the 8 warps)
-            auto exchange = [&](float v, float &other) -> bool {
-                const int buf = x_x & 1;
-                xchg_sh[buf][hf][r] = v;
-                tc_fence_before();  // this warp's tensor-memory reads happen before the arrival
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&xbar);
-                if (!mbar_wait_warp(&xbar, x_x & 1, &abort_sh, a.err, lim_ns)) return false;
-                tc_fence_after();
-                other = xchg_sh[buf][hf ^ 1][r];
-                ++x_x;
-                return true;
-            };
             for (int si = 0; si < nseg && ok; ++si) {
                 const Seg sg = segs[si];
                 const int b = sg.b;
                 const int T = clamp_len(__ldg(a.seqlens + b), max_tokens, a.L, nullptr);
                 const int lim = row_ok ? T - a.L + i_row : -1;
-                if (hf == 0) {
+                {
                     // q's latent part of this segment's rows -> tensor memory (the A operand of
                     // the score product), once the previous segment's score MMAs are done with it
                     if (!mbar_wait_warp(&qempty_bar, (x_q & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
@@ -336,35 +324,30 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 ++x_q;
                 // l: sum of the fp32 P (gives lse); lq: sum of the bf16-rounded P the product
-                // uses (normalises O: a convex combination of the rounded weights).  Both are
-                // partial over this thread's columns until the epilogue.
+                // uses (normalises O: a convex combination of the rounded weights).
                 float m_ref = -INFINITY, l = 0.f, lq = 0.f;
                 for (int tile = sg.t0; tile < sg.t1; ++tile) {
-                    const int tok0 = tile * TOK + hf * HC;       // first token of this thread's columns
+                    const int tok0 = tile * TOK;
                     const uint32_t sb = x_s & 1;
                     if (!mbar_wait_warp(&sfull_bar[sb], (x_s >> 1) & 1, &abort_sh, a.err, lim_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    float s[HC];
+                    float s[TOK];
                     float mx = -INFINITY;
                     if (warp_live) {
-                        if constexpr (HC == 32) {
-                            tmem_ld32(tmem + lane_base + C::S_COL + sb * TOK + hf * HC, s);
-                        } else {
-                            tmem_ld16(tmem + lane_base + C::S_COL + sb * TOK + hf * HC, s);
+#pragma unroll
+                        for (int h = 0; h < TOK / 32; ++h) {
+                            float t32[32];
+                            tmem_ld32(tmem + lane_base + C::S_COL + sb * TOK + 32 * h, t32);
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) s[32 * h + k] = t32[k];
                         }
                     }
                     ++x_s;
                     const bool full = tile * TOK + TOK - 1 <= T - a.L && row_ok;  // no column masked
                     if (warp_live) mx = tile_max(s, full, tok0, lim, a.scale_log2);
-                    float mo;
-                    if (!exchange(mx, mo)) {
-                        ok = false;
-                        break;
-                    }
-                    mx = fmaxf(mx, mo);
                     float alpha = 1.f;
                     bool need = false;
                     if (mx != -INFINITY) {
@@ -386,13 +369,12 @@ __global__ void __launch_bounds__(384, 1)
                         l *= alpha;
                         lq *= alpha;
 #pragma unroll 1
-                        for (int ch = 0; ch < DV / 64; ++ch) {
+                        for (int ch = 0; ch < DV / 32; ++ch) {
                             float o[32];
-                            const uint32_t col = hf * (DV / 2) + ch * 32;
-                            tmem_ld32(tmem + lane_base + col, o);
+                            tmem_ld32(tmem + lane_base + ch * 32, o);
 #pragma unroll
                             for (int k = 0; k < 32; ++k) o[k] *= alpha;
-                            tmem_st32(tmem + lane_base + col, o);
+                            tmem_st32(tmem + lane_base + ch * 32, o);
                         }
                         tmem_st_wait();
                     }
@@ -406,27 +388,25 @@ __global__ void __launch_bounds__(384, 1)
                         const int k0 = max(T - ttok0, 0);
                         uint8_t *v0 = stage_s + (size_t)stage * C::STAGE + (size_t)vc * 4 * C::CHUNK;
                         const int units = (TOK - k0) * 4 * 8;  // 16-byte units: rows x 4 chunks x 8
-                        for (int u = st_id; u < units; u += 256) {
+                        for (int u = st_id; u < units; u += 32 * NSMX) {
                             const int row = k0 + u / 32, ch = (u / 8) & 3, k = u & 7;
                             *(uint4 *)(v0 + ch * C::CHUNK + row * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                         }
                     }
-                    // P (bf16 pairs) over S in buffer x_pv & 1: both halves have read their S
-                    // columns (the row-max exchange above orders that)
+                    // P (bf16 pairs) over S in buffer x_pv & 1 (this thread has read its S row)
                     if (warp_live) {
-                        const uint32_t pa = tmem + lane_base + C::S_COL + sb * TOK + hf * (HC / 2);
-                        uint32_t w[HC / 2];
+                        const uint32_t pa = tmem + lane_base + C::S_COL + sb * TOK;
                         float sum = 0.f, sum2 = 0.f;
 #pragma unroll
-                        for (int k = 0; k < HC / 2; ++k) {
-                            w[k] = pack_bf16(s[2 * k], s[2 * k + 1]);
-                            sum += bf16_lo(w[k]);
-                            sum2 += bf16_hi(w[k]);
-                        }
-                        if constexpr (HC == 32) {
-                            tmem_st16u(pa, w);
-                        } else {
-                            tmem_st8u(pa, w);
+                        for (int h = 0; h < TOK / 32; ++h) {
+                            uint32_t w[16];
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) {
+                                w[k] = pack_bf16(s[32 * h + 2 * k], s[32 * h + 2 * k + 1]);
+                                sum += bf16_lo(w[k]);
+                                sum2 += bf16_hi(w[k]);
+                            }
+                            tmem_st16u(pa + 16 * h, w);
                         }
                         tmem_st_wait();
                         lq += sum + sum2;
@@ -440,14 +420,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 if (!ok) break;
 
-                // ---- epilogue: merge the two halves' sums; O is final once the last P.V completes
-                float lo, lqo;
-                if (!exchange(l, lo) || !exchange(lq, lqo)) {
-                    ok = false;
-                    break;
-                }
-                l += lo;
-                lq += lqo;
+                // ---- epilogue: O is final once the last P.V completes
                 if (!wait_pv(x_pv - 1)) {
                     ok = false;
                     break;
@@ -459,9 +432,9 @@ __global__ void __launch_bounds__(384, 1)
                 const size_t r_out = (size_t)i_row * a.h_q + head;
                 if (warp_live) {
 #pragma unroll 1
-                    for (int ch = 0; ch < DV / 64; ++ch) {
+                    for (int ch = 0; ch < DV / 32; ++ch) {
                         float o[32];
-                        const int col = hf * (DV / 2) + ch * 32;
+                        const int col = ch * 32;
                         tmem_ld32(tmem + lane_base + col, o);
                         if (!row_ok) continue;
                         if (sg.nsplit == 1) {
@@ -482,7 +455,7 @@ __global__ void __launch_bounds__(384, 1)
                         }
                     }
                 }
-                if (row_ok && vc == 0 && hf == 0) {
+                if (row_ok && vc == 0) {
                     if (sg.nsplit == 1)
                         a.lse[(size_t)b * rows_b + r_out] = lse_v;
                     else
@@ -514,7 +487,7 @@ cudaError_t launch_t(const CUtensorMap &qm, const CUtensorMap &lm, const CUtenso
     auto k = latent_decode_kernel<DC, TOK>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, 384, smem, st>>>(qm, lm, rm, a);
+    k<<<grid, LTHREADS, smem, st>>>(qm, lm, rm, a);
     return cudaGetLastError();
 }
 
