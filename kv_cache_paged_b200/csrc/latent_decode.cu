@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     using C = LatCfg<DC, TOK>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
-    __shared__ uint64_t qfull_bar, qtm_bar, qempty_bar, sfull_bar[2], pfull_bar[2], pfree_bar[2], end_bar;
+    __shared__ uint64_t qfull_bar, qtm_bar, qempty_bar, sfull_bar[2], pfull_bar[2], end_bar;
     __shared__ Seg segs[LMAXSEG];
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
@@ -95,7 +95,6 @@ __global__ void __launch_bounds__(LTHREADS, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sfull_bar[s], 1);
             mbar_init(&pfull_bar[s], NSMX);  // one arrival per softmax warp
-            mbar_init(&pfree_bar[s], 1);
         }
         mbar_init(&end_bar, 1);
         abort_sh = 0;
@@ -260,8 +259,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                         for (int kk = 0; kk < TOK / 16; ++kk)
                             umma_bf16_ts(tmem, pa + kk * 8, dv0 + (uint64_t)(kk * 128), idesc_pv,
                                          (j > 0 || kk > 0) ? 1u : 0u);
-                        umma_commit(&pfree_bar[pb]);
-                        umma_commit(&empty_bar[stage]);
+                        umma_commit(&empty_bar[stage]);  // the stage is free and P.V j is done
                         ++m_pv;
                     }
                     m_tile += n;
@@ -285,9 +283,11 @@ __global__ void __launch_bounds__(LTHREADS, 1)
             const int i_row = row_ok ? n_row / g : 0;
             const int head = row_ok ? c * g + n_row % g : 0;
             bool ok = true;
-            // wait until P.V number k has completed (it frees P buffer k & 1 and settles O)
+            // wait until P.V number k has completed (O settled): the commit that frees tile k's
+            // stage.  Every earlier P.V is complete by then (P(k) needed S(k), issued after P.V
+            // k - 2), so the barrier is at most one phase short of the one waited for.
             auto wait_pv = [&](uint32_t k) -> bool {
-                return mbar_wait_warp(&pfree_bar[k & 1], (k >> 1) & 1, &abort_sh, a.err, lim_ns);
+                return mbar_wait_warp(&empty_bar[k % nstage], (k / nstage) & 1, &abort_sh, a.err, lim_ns);
             };
             for (int si = 0; si < nseg && ok; ++si) {
                 const Seg sg = segs[si];

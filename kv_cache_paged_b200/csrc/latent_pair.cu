@@ -14,9 +14,9 @@
 //
 // Roles per CTA: warps 0..3 send (one per TMEM lane quadrant: write q's latent half into tensor
 // memory at the start of each sequence, then per tile load this CTA's partial S and bulk-copy it
-// into the peer's receive buffer, one 32-token half at a time), warps 4..11 softmax (two threads
-// per row, one per 32-token half of the tile; each adds the peer's partial from its receive
-// buffer to its own from tensor memory), warp 12 TMA producer, warp 13 MMA issuer (one thread).
+// into the peer's receive buffer, one 32-token half at a time), warps 4..7 softmax (one thread
+// per row: it adds the peer's partial from the receive buffer to its own from tensor memory),
+// warp 8 TMA producer, warp 9 MMA issuer (one thread).
 // Tensor memory: O [0, 256), two S buffers [256, 384) with P(j) written over S(j) as bf16 pairs,
 // and q's latent half [384, 512) as the A operand of the score product.  Keeping q there leaves
 // shared memory for four 36 KB KV stages next to the exchange buffers.  Every wait is bounded.
@@ -41,23 +41,24 @@ constexpr uint32_t P_XBYTES = 4 * P_XHALF;                // send and receive bu
 constexpr int P_NSB = 2;                                  // S buffers (P is written over its S)
 constexpr uint32_t P_SCOL = PDV;                          // S buffers [256, 384)
 constexpr uint32_t P_QCOL = PDV + P_NSB * PTOK;           // q latent half [384, 512), bf16 pairs
-constexpr int W_PROD = 12, W_MMA = 13;
+constexpr int P_NSMX = 4;                                 // softmax warps, one thread per row
+constexpr int W_PROD = 4 + P_NSMX, W_MMA = 5 + P_NSMX;
+constexpr int P_THREADS = 32 * (6 + P_NSMX);
 constexpr float P_RESCALE_LOG2 = 8.f;
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     mla_pair_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap qrmap,
                     const __grid_constant__ CUtensorMap latmap, const __grid_constant__ CUtensorMap ropemap,
                     const LatentArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
-    __shared__ uint64_t qfull_bar, qtm_bar, qempty_bar, pfull_bar[P_NSB], pfree_bar[P_NSB], end_bar;
+    __shared__ uint64_t qfull_bar, qtm_bar, qempty_bar, pfull_bar[P_NSB], end_bar;
     __shared__ uint64_t sfull_bar[P_NSB], sread_bar[P_NSB];
-    __shared__ uint64_t xbar, xfull_bar[2], xfree_bar[2];
+    __shared__ uint64_t xfull_bar[2], xfree_bar[2];
     __shared__ Seg segs[PMAXSEG];
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
     __shared__ uint32_t tmem_sh;
-    __shared__ float xchg_sh[2][2][128];
 
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *q_s = smem;
@@ -87,21 +88,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         mbar_init(&qtm_bar, 4);     // q latent half written into tensor memory by the send warps
         mbar_init(&qempty_bar, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&pfull_bar[s], 8);
-            mbar_init(&pfree_bar[s], 1);
+            mbar_init(&pfull_bar[s], P_NSMX);
         }
         for (int s = 0; s < P_NSB; ++s) {
             mbar_init(&sfull_bar[s], 1);    // partial S computed (MMA commit)
             mbar_init(&sread_bar[s], 4);    // partial S read by the send warps (P may overwrite it)
         }
         mbar_init(&end_bar, 1);
-        mbar_init(&xbar, 8);
         // per 32-token half h of a tile: xfull[h] takes one local arrival that arms the expected
         // bytes and is completed by the peer's bulk copies (16 KB); xfree[h] takes one arrival
-        // from each of the peer's 4 softmax warps that read half h
+        // from each of the peer's softmax warps
         for (int h = 0; h < 2; ++h) {
             mbar_init(&xfull_bar[h], 1);
-            mbar_init(&xfree_bar[h], 4);
+            mbar_init(&xfree_bar[h], P_NSMX);
             mbar_arrive_expect_tx(&xfull_bar[h], P_XHALF);  // armed for the first tile
         }
         abort_sh = 0;
@@ -121,7 +120,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
 
     uint32_t p_issued = 0, p_qloads = 0;
     uint32_t m_tile = 0, m_q = 0;
-    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0;   // softmax
+    uint32_t x_tile = 0, x_s = 0, x_pv = 0;            // softmax
     uint32_t e_t = 0, e_q = 0;                          // send
 
     for (int skip = 0;; skip += PMAXSEG) {
@@ -261,7 +260,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                         for (int kk = 0; kk < PTOK / 16; ++kk)
                             umma_bf16_ts(tmem, pa + kk * 8, dv0 + (uint64_t)(kk * 128), idesc_pv,
                                          (j > 0 || kk > 0) ? 1u : 0u);
-                        umma_commit(&pfree_bar[pb]);
                         umma_commit(&empty_bar[stage]);
                     }
                     m_tile += n;
@@ -350,35 +348,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                     }
                 }
             }
-        } else if (warp >= 4 && warp < 12) {
+        } else if (warp >= 4 && warp < 4 + P_NSMX) {
             // ================================================================ softmax / epilogue
-            constexpr int HC = PTOK / 2;
+            // One thread per row (TMEM lane): the whole 64-token S row, so no row value crosses
+            // threads.  The peer's partial arrives in two 32-token halves.
             const int st_id = threadIdx.x - 128;
-            const int hf = (warp - 4) >> 2;
             const int r = (warp & 3) * 32 + lane;
             const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
             const int n_row = rt * 128 + r;
             const bool row_ok = n_row < R;
             const bool warp_live = rt * 128 + (warp & 3) * 32 < R;
             const uint32_t peer_xfree[2] = {mapa_shared(smem_u32(&xfree_bar[0]), peer),
-                                                mapa_shared(smem_u32(&xfree_bar[1]), peer)};
+                                            mapa_shared(smem_u32(&xfree_bar[1]), peer)};
             const int i_row = row_ok ? n_row / g : 0;
             const int head = row_ok ? c * g + n_row % g : 0;
             bool ok = true;
+            // P.V number k has completed (O settled): the commit that frees tile k's stage.  Every
+            // earlier P.V is complete by then (P(k) needed S(k), issued after P.V k - 2), so the
+            // barrier is at most one phase short of the one waited for.
             auto wait_pv = [&](uint32_t k) -> bool {
-                return mbar_wait_warp(&pfree_bar[k & 1], (k >> 1) & 1, &abort_sh, a.err, lim_ns);
-            };
-            auto exchange = [&](float v, float &other) -> bool {
-                const int buf = x_x & 1;
-                xchg_sh[buf][hf][r] = v;
-                tc_fence_before();  // this warp's tensor-memory reads happen before the arrival
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&xbar);
-                if (!mbar_wait_warp(&xbar, x_x & 1, &abort_sh, a.err, lim_ns)) return false;
-                tc_fence_after();
-                other = xchg_sh[buf][hf ^ 1][r];
-                ++x_x;
-                return true;
+                return mbar_wait_warp(&empty_bar[k % nstage], (k / nstage) & 1, &abort_sh, a.err, lim_ns);
             };
             for (int si = 0; si < nseg && ok; ++si) {
                 const Seg sg = segs[si];
@@ -387,25 +376,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                 const int lim = row_ok ? T - a.L + i_row : -1;
                 float m_ref = -INFINITY, l = 0.f, lq = 0.f;
                 for (int tile = sg.t0; tile < sg.t1; ++tile) {
-                    const int tok0 = tile * PTOK + hf * HC;
+                    const int tok0 = tile * PTOK;
                     const uint32_t sb = x_s % P_NSB;
                     if (!mbar_wait_warp(&sfull_bar[sb], (x_s / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    float s[HC];
-                    tmem_ld32(tmem + lane_base + P_SCOL + sb * PTOK + hf * HC, s);
+                    float s[PTOK];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float t32[32];
+                        tmem_ld32(tmem + lane_base + P_SCOL + sb * PTOK + 32 * h, t32);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) s[32 * h + k] = t32[k];
+                    }
                     // S = own partial + the peer's (the peer adds in the opposite order; fp32
                     // addition commutes, so both CTAs see the same S bit for bit)
-                    if (!mbar_wait_warp_cluster(&xfull_bar[hf], x_s & 1, &abort_sh, a.err, lim_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    // the phase is complete: arm the next tile's before any warp releases the buffer
-                    if (threadIdx.x == 128 + 128 * hf) mbar_arrive_expect_tx(&xfull_bar[hf], P_XHALF);
-                    {
-                        const uint32_t row = smem_u32(recv_s + hf * P_XHALF) + r * 128;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (!mbar_wait_warp_cluster(&xfull_bar[h], x_s & 1, &abort_sh, a.err, lim_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        // the phase is complete: arm the next tile's before any warp frees the buffer
+                        if (threadIdx.x == 128) mbar_arrive_expect_tx(&xfull_bar[h], P_XHALF);
+                        const uint32_t row = smem_u32(recv_s + h * P_XHALF) + r * 128;
 #pragma unroll
                         for (int c8 = 0; c8 < 8; ++c8) {
                             float4 v;
@@ -413,25 +409,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                                          : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                                          : "r"(row + ((c8 ^ (r & 7)) << 4))
                                          : "memory");
-                            s[4 * c8] += v.x;
-                            s[4 * c8 + 1] += v.y;
-                            s[4 * c8 + 2] += v.z;
-                            s[4 * c8 + 3] += v.w;
+                            s[32 * h + 4 * c8] += v.x;
+                            s[32 * h + 4 * c8 + 1] += v.y;
+                            s[32 * h + 4 * c8 + 2] += v.z;
+                            s[32 * h + 4 * c8 + 3] += v.w;
                         }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(peer_xfree[h]);
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(peer_xfree[hf]);
+                    if (!ok) break;
                     ++x_s;
 
                     float mx = -INFINITY;
                     const bool full = tile * PTOK + PTOK - 1 <= T - a.L && row_ok;  // no column masked
                     if (warp_live) mx = tile_max(s, full, tok0, lim, a.scale_log2);
-                    float mo;
-                    if (!exchange(mx, mo)) {
-                        ok = false;
-                        break;
-                    }
-                    mx = fmaxf(mx, mo);
                     float alpha = 1.f;
                     bool need = false;
                     if (mx != -INFINITY) {
@@ -452,13 +443,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                         l *= alpha;
                         lq *= alpha;
 #pragma unroll 1
-                        for (int ch = 0; ch < PDV / 64; ++ch) {
+                        for (int ch = 0; ch < PDV / 32; ++ch) {
                             float o[32];
-                            const uint32_t col = hf * (PDV / 2) + ch * 32;
-                            tmem_ld32(tmem + lane_base + col, o);
+                            tmem_ld32(tmem + lane_base + ch * 32, o);
 #pragma unroll
                             for (int k = 0; k < 32; ++k) o[k] *= alpha;
-                            tmem_st32(tmem + lane_base + col, o);
+                            tmem_st32(tmem + lane_base + ch * 32, o);
                         }
                         tmem_st_wait();
                     }
@@ -470,29 +460,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                         const int k0 = max(T - ttok0, 0);
                         uint8_t *v0 = stage_s + (size_t)stage * P_STAGE;
                         const int units = (PTOK - k0) * 4 * 8;
-                        for (int u = st_id; u < units; u += 256) {
+                        for (int u = st_id; u < units; u += 32 * P_NSMX) {
                             const int row = k0 + u / 32, ch = (u / 8) & 3, k = u & 7;
                             *(uint4 *)(v0 + ch * P_CHUNK + row * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                         }
                     }
-                    // P(j) is written over S(j): both warpgroups have read their S columns (the
-                    // row-max exchange above orders that) and the send warps must have too
+                    // P(j) is written over S(j): the send warps must have read it too
                     if (!mbar_wait_warp(&sread_bar[sb], (x_pv / P_NSB) & 1, &abort_sh, a.err, lim_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     if (warp_live) {
-                        const uint32_t pa = tmem + lane_base + P_SCOL + sb * PTOK + hf * (HC / 2);
-                        uint32_t w[HC / 2];
+                        const uint32_t pa = tmem + lane_base + P_SCOL + sb * PTOK;
                         float sum = 0.f, sum2 = 0.f;
 #pragma unroll
-                        for (int k = 0; k < HC / 2; ++k) {
-                            w[k] = pack_bf16(s[2 * k], s[2 * k + 1]);
-                            sum += bf16_lo(w[k]);
-                            sum2 += bf16_hi(w[k]);
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t w[16];
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) {
+                                w[k] = pack_bf16(s[32 * h + 2 * k], s[32 * h + 2 * k + 1]);
+                                sum += bf16_lo(w[k]);
+                                sum2 += bf16_hi(w[k]);
+                            }
+                            tmem_st16u(pa + 16 * h, w);
                         }
-                        tmem_st16u(pa, w);
                         tmem_st_wait();
                         lq += sum + sum2;
                     }
@@ -505,13 +497,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                 }
                 if (!ok) break;
 
-                float lo, lqo;
-                if (!exchange(l, lo) || !exchange(lq, lqo)) {
-                    ok = false;
-                    break;
-                }
-                l += lo;
-                lq += lqo;
                 if (!wait_pv(x_pv - 1)) {
                     ok = false;
                     break;
@@ -523,9 +508,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                 const size_t r_out = (size_t)i_row * a.h_q + head;
                 if (warp_live) {
 #pragma unroll 1
-                    for (int ch = 0; ch < PDV / 64; ++ch) {
+                    for (int ch = 0; ch < PDV / 32; ++ch) {
                         float o[32];
-                        const int col = hf * (PDV / 2) + ch * 32;
+                        const int col = ch * 32;
                         tmem_ld32(tmem + lane_base + col, o);
                         if (!row_ok) continue;
                         const int gcol = kr * PDV + col;
@@ -546,7 +531,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                         }
                     }
                 }
-                if (row_ok && kr == 0 && hf == 0) {
+                if (row_ok && kr == 0) {
                     if (sg.nsplit == 1)
                         a.lse[(size_t)b * rows_b + r_out] = lse_v;
                     else
@@ -581,7 +566,7 @@ cudaError_t launch_mla_pair(const CUtensorMap &qm, const CUtensorMap &qrm, const
                             const CUtensorMap &rm, const LatentArgs &a, int grid, size_t smem, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(mla_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    mla_pair_kernel<<<grid, 448, smem, st>>>(qm, qrm, lm, rm, a);
+    mla_pair_kernel<<<grid, P_THREADS, smem, st>>>(qm, qrm, lm, rm, a);
     return cudaGetLastError();
 }
 
