@@ -53,8 +53,10 @@ def describe(inp):
         kind, shape = "GTA", f"h_q {inp.h_q}, h_kv {inp.h_kv}, d_h {inp.d}, d_r {inp.d_r}"
     else:
         kind, shape = "GQA", f"h_q {inp.h_q}, h_kv {inp.h_kv}, d {inp.d}"
+    pre = (f", the first {inp.shared_prefix} tokens a prefix shared by the batch (stored once; "
+           f"algorithmic bytes count it once)") if getattr(inp, "shared_prefix", 0) else ""
     return (f"{kind} paged decode: B {inp.B}, q_len {inp.L}, {shape}, page {inp.page_size}, "
-            f"contexts {int(sl.min())}..{int(sl.max())} (mean {float(sl.mean()):.0f})")
+            f"contexts {int(sl.min())}..{int(sl.max())} (mean {float(sl.mean()):.0f}){pre}")
 
 
 def load_peaks():
@@ -375,7 +377,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="kvd", choices=["kvd", "reference"])
-    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny"] + list(APPEND_SHAPES))
+    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny", "gta_prefix"] + list(APPEND_SHAPES))
     ap.add_argument("--tokens", type=int, default=65536, help="new tokens per call (append workloads)")
     ap.add_argument("--qlen", type=int, default=1)
     ap.add_argument("--page-size", type=int, default=0, help="override the workload's page size (tokens per page)")

@@ -172,6 +172,21 @@ int kvd_gla_decode(const kvd_gla_params *p, void *workspace, size_t workspace_by
 int kvd_gta_decode_noalloc(const kvd_gta_params *p, kvd_stream_t stream);
 
 /*
+ * Merge two attention states of the same query rows over disjoint key sets, e.g. a prefix
+ * shared by the whole batch and each sequence's own continuation (cascade decoding; the
+ * combine step of "Hardware-Efficient Attention for Fast Decoding", section 3.3.2, applied
+ * to two parts).  With m = max(lse_a, lse_b):
+ *   lse = m + ln(e^(lse_a - m) + e^(lse_b - m)),
+ *   out = e^(lse_a - lse) out_a + e^(lse_b - lse) out_b,
+ * a state with lse = -inf weighs nothing, and two empty states give out = 0, lse = -inf.
+ * out_a, out_b, out: bf16 [rows, d_v] (device, 16-byte aligned, d_v a multiple of 8);
+ * lse_a, lse_b, lse: fp32 [rows] (device).  out / lse may be out_a / lse_a (in place).
+ * Arithmetic in fp32, out rounded to bf16.  Asynchronous on `stream`.
+ */
+int kvd_merge_states(const void *out_a, const float *lse_a, const void *out_b, const float *lse_b, void *out,
+                     float *lse, int32_t rows, int32_t d_v, kvd_stream_t stream);
+
+/*
  * Split plan for inspection and tests.  Cuts the (sequence, tile) stream of
  * seqlens[B] (device pointer) with `tile` tokens per tile into num_parts parts
  * exactly as the decode kernels do and writes, for part c, up to `cap` records

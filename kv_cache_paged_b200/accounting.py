@@ -52,11 +52,17 @@ def step_flops(variant, seqlens, *, L, h_q, d, d_r) -> int:
 
 
 def of_inputs(inp):
-    """(bytes, flops, kv_bytes) for a decode-inputs record."""
+    """(bytes, flops, kv_bytes) for a decode-inputs record.  A prefix shared by the batch
+    (stored once) is algorithmically read once: its tokens count once, not once per sequence."""
     kw = dict(L=inp.L, h_q=inp.h_q, h_kv=inp.h_kv, d=inp.d, d_r=inp.d_r, page_size=inp.page_size)
     b = step_bytes(inp.variant, inp.seqlens, **kw)
     f = step_flops(inp.variant, inp.seqlens, L=inp.L, h_q=inp.h_q, d=inp.d, d_r=inp.d_r)
-    return b, f, kv_bytes(inp.variant, inp.seqlens, inp.h_kv, inp.d, inp.d_r)
+    kvb = kv_bytes(inp.variant, inp.seqlens, inp.h_kv, inp.d, inp.d_r)
+    shared = getattr(inp, "shared_prefix", 0)
+    if shared and inp.B > 1:
+        dup = (inp.B - 1) * shared * kv_elems_per_token(inp.variant, inp.h_kv, inp.d, inp.d_r) * 2
+        b, kvb = b - dup, kvb - dup
+    return b, f, kvb
 
 
 def roofline_us(nbytes: float, flops: float, hbm_gbs: float, tflops: float) -> float:

@@ -115,6 +115,8 @@ def lib():
                 f = getattr(L, f"kvd_{name}_append")
                 f.restype = ctypes.c_int
                 f.argtypes = [ctypes.POINTER(P), _vp]
+            L.kvd_merge_states.restype = ctypes.c_int
+            L.kvd_merge_states.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp]
             L.kvd_rope_q.restype = ctypes.c_int
             L.kvd_rope_q.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, ctypes.c_float, _vp]
             _lib = L
@@ -370,3 +372,21 @@ def rope_q(q, seqlens, rope_off, d_r, *, rope_base=10000.0, stream=None):
     st = lib().kvd_rope_q(_dev(q, "q", torch.bfloat16, 4), _dev(seqlens, "seqlens", torch.int32, 1), B, L, heads,
                           d_qk, rope_off, d_r, rope_base, _stream_ptr(stream))
     _check("kvd_rope_q", st)
+
+
+# ----------------------------------------------------------------------------- cascade
+def merge_states(out_a, lse_a, out_b, lse_b, *, out=None, lse=None, stream=None):
+    """Merge two attention states (out bf16 [..., d_v], lse fp32 [...]) over disjoint key sets."""
+    torch = _torch()
+    if out_a.shape != out_b.shape or lse_a.shape != lse_b.shape or out_a.shape[:-1] != lse_a.shape:
+        raise ValueError("states must have matching shapes")
+    d_v = out_a.shape[-1]
+    rows = lse_a.numel()
+    out = torch.empty_like(out_a) if out is None else out
+    lse = torch.empty_like(lse_a) if lse is None else lse
+    st = lib().kvd_merge_states(_dev(out_a, "out_a", torch.bfloat16), _dev(lse_a, "lse_a", torch.float32),
+                                _dev(out_b, "out_b", torch.bfloat16), _dev(lse_b, "lse_b", torch.float32),
+                                _dev(out, "out", torch.bfloat16), _dev(lse, "lse", torch.float32), rows, d_v,
+                                _stream_ptr(stream))
+    _check("kvd_merge_states", st)
+    return out, lse

@@ -450,6 +450,18 @@ int kvd_gta_decode(const kvd_gta_params *p, void *ws, size_t ws_bytes, kvd_strea
                      p->num_parts, ws, ws_bytes, (cudaStream_t)stream);
 }
 
+int kvd_merge_states(const void *out_a, const float *lse_a, const void *out_b, const float *lse_b, void *out,
+                     float *lse, int32_t rows, int32_t d_v, kvd_stream_t stream) {
+    if (rows < 0 || d_v <= 0 || d_v % 8) return KVD_ERR_INVALID_ARG;
+    if (!out_a || !out_b || !out || !lse_a || !lse_b || !lse) return KVD_ERR_INVALID_ARG;
+    if (!aligned(out_a, 16) || !aligned(out_b, 16) || !aligned(out, 16) || !aligned(lse_a, 4) || !aligned(lse_b, 4) ||
+        !aligned(lse, 4))
+        return KVD_ERR_INVALID_ARG;
+    return launch_merge(out_a, lse_a, out_b, lse_b, out, lse, rows, d_v, (cudaStream_t)stream) == cudaSuccess
+               ? KVD_OK
+               : KVD_ERR_CUDA;
+}
+
 int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_tokens, int32_t num_parts,
              int32_t *segments, int32_t *counts, int32_t cap, kvd_stream_t stream) {
     if (B < 0 || tile < 1 || max_tokens < 0 || num_parts < 1 || cap < 0) return KVD_ERR_INVALID_ARG;

@@ -125,7 +125,53 @@ __global__ void plan_kernel(const int32_t *seqlens, int B, int tile, int max_tok
     if ((threadIdx.x & 31) == 0) counts[c] = cnt;
 }
 
+// Merge two attention states over disjoint key sets of the same query rows (a shared
+// prefix and a sequence's own continuation): with m = max(lse_a, lse_b),
+// lse = m + ln(e^(lse_a - m) + e^(lse_b - m)) and out = e^(lse_a - lse) out_a + e^(lse_b - lse) out_b.
+// A state with lse = -inf (no key) has weight 0; two empty states give out = 0, lse = -inf.
+// One thread per 8 output elements (16 bytes of bf16).
+__global__ void __launch_bounds__(256) merge_kernel(const __nv_bfloat16 *out_a, const float *lse_a,
+                                                    const __nv_bfloat16 *out_b, const float *lse_b,
+                                                    __nv_bfloat16 *out, float *lse, int rows, int d_v) {
+    const int per_row = d_v / 8;
+    const long long u = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (u >= (long long)rows * per_row) return;
+    const int row = (int)(u / per_row), k = (int)(u % per_row);
+    const float la = __ldg(lse_a + row), lb = __ldg(lse_b + row);
+    const float m = fmaxf(la, lb);
+    float wa = 0.f, wb = 0.f, l = -INFINITY;
+    if (m != -INFINITY) {
+        const float ea = expf(la - m), eb = expf(lb - m);
+        const float inv = 1.f / (ea + eb);
+        wa = ea * inv;
+        wb = eb * inv;
+        l = m + logf(ea + eb);
+    }
+    const uint4 va = __ldg((const uint4 *)(out_a + (size_t)row * d_v) + k);
+    const uint4 vb = __ldg((const uint4 *)(out_b + (size_t)row * d_v) + k);
+    const uint32_t xa[4] = {va.x, va.y, va.z, va.w}, xb[4] = {vb.x, vb.y, vb.z, vb.w};
+    uint32_t y[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        // a state of weight 0 contributes nothing (its out may hold anything, e.g. zeros)
+        const float lo = (wa > 0.f ? wa * bf16_lo(xa[i]) : 0.f) + (wb > 0.f ? wb * bf16_lo(xb[i]) : 0.f);
+        const float hi = (wa > 0.f ? wa * bf16_hi(xa[i]) : 0.f) + (wb > 0.f ? wb * bf16_hi(xb[i]) : 0.f);
+        y[i] = pack_bf16(lo, hi);
+    }
+    *((uint4 *)(out + (size_t)row * d_v) + k) = make_uint4(y[0], y[1], y[2], y[3]);
+    if (k == 0) lse[row] = l;
+}
+
 }  // namespace
+
+cudaError_t launch_merge(const void *out_a, const float *lse_a, const void *out_b, const float *lse_b, void *out,
+                         float *lse, int rows, int d_v, cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    const long long units = (long long)rows * (d_v / 8);
+    merge_kernel<<<(unsigned)((units + 255) / 256), 256, 0, st>>>(
+        (const __nv_bfloat16 *)out_a, lse_a, (const __nv_bfloat16 *)out_b, lse_b, (__nv_bfloat16 *)out, lse, rows, d_v);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
     if (a.B == 0 || a.rows == 0) return cudaSuccess;

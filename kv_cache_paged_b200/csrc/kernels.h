@@ -90,6 +90,10 @@ struct CombineArgs {
     int d_v;
 };
 
+// Merges two attention states (out bf16 [rows, d_v], lse fp32 [rows]) over disjoint key sets.
+cudaError_t launch_merge(const void *out_a, const float *lse_a, const void *out_b, const float *lse_b, void *out,
+                         float *lse, int rows, int d_v, cudaStream_t st);
+
 // Merges split partials (launched as a programmatic dependent of the decode kernel).
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 

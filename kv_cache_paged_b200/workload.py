@@ -35,7 +35,7 @@ import numpy as np
 BF16_NAN = np.uint16(0x7FC0)
 
 # Seeds per named workload.
-SEEDS = {"gta_tiny": 0, "gta": 1, "gqa": 2, "mla": 3, "gla2": 4}
+SEEDS = {"gta_tiny": 0, "gta": 1, "gqa": 2, "mla": 3, "gla2": 4, "gta_prefix": 5}
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -74,6 +74,7 @@ class DecodeInputs:
     caches: dict = field(default_factory=dict)   # name -> uint16 array
     poison_page: int = -1
     name: str = ""
+    shared_prefix: int = 0  # tokens at the start of every sequence stored once, in shared pages
 
     @property
     def d_qk(self) -> int:
@@ -123,19 +124,25 @@ def draw_seqlens(rng: np.random.Generator, B: int, spec, L: int = 1) -> np.ndarr
     return arr
 
 
-def make_paging(rng: np.random.Generator, seqlens: np.ndarray, page_size: int, shuffle: bool = True):
-    """Block table over a pool of sum ceil(T_b/S) used pages plus one unreferenced page."""
+def make_paging(rng: np.random.Generator, seqlens: np.ndarray, page_size: int, shuffle: bool = True,
+                prefix_pages: int = 0):
+    """Block table over a pool of the used pages plus one unreferenced page.  The first
+    ``prefix_pages`` logical pages of every sequence are the same physical pages (a prefix
+    shared by the whole batch, stored once); the other pages belong to one sequence each."""
     B = len(seqlens)
     npages = [(int(t) + page_size - 1) // page_size for t in seqlens]
-    used = sum(npages)
+    assert all(n > prefix_pages for n in npages) or prefix_pages == 0, "sequences must extend past the prefix"
+    own = [n - prefix_pages for n in npages]
+    used = prefix_pages + sum(own)
     max_pages = max(1, max(npages) if npages else 1)
     num_pages = used + 1
     perm = rng.permutation(num_pages).astype(np.int32) if shuffle else np.arange(num_pages, dtype=np.int32)
     table = np.full((B, max_pages), -1, dtype=np.int32)
-    k = 0
+    k = prefix_pages
     for b in range(B):
-        table[b, : npages[b]] = perm[k: k + npages[b]]
-        k += npages[b]
+        table[b, :prefix_pages] = perm[:prefix_pages]
+        table[b, prefix_pages: npages[b]] = perm[k: k + own[b]]
+        k += own[b]
     poison = int(perm[used])
     return table, num_pages, max_pages, poison
 
@@ -152,12 +159,16 @@ def poison_cache(cache: np.ndarray, seqlens: np.ndarray, table: np.ndarray, pois
 
 def make_inputs(variant: str, *, B: int, L: int, h_q: int, h_kv: int, d: int, d_r: int = 0,
                 page_size: int, seqlens, seed: int, scale: float | None = None,
-                latent_scale: float = 1.0, shuffle: bool = True, name: str = "") -> DecodeInputs:
-    """Draw a full decode step for ``variant`` in ("gqa", "gta", "gla")."""
+                latent_scale: float = 1.0, shuffle: bool = True, name: str = "",
+                shared_prefix: int = 0) -> DecodeInputs:
+    """Draw a full decode step for ``variant`` in ("gqa", "gta", "gla").  With
+    ``shared_prefix`` (a multiple of the page size) every sequence starts with the same
+    ``shared_prefix`` tokens, stored once; ``seqlens`` then draws the lengths past it."""
     assert variant in ("gqa", "gta", "gla")
+    assert shared_prefix % page_size == 0, "the shared prefix covers whole pages"
     rng = np.random.default_rng(seed)
-    sl = draw_seqlens(rng, B, seqlens, L)
-    table, num_pages, max_pages, poison = make_paging(rng, sl, page_size, shuffle)
+    sl = (draw_seqlens(rng, B, seqlens, L) + shared_prefix).astype(np.int32)
+    table, num_pages, max_pages, poison = make_paging(rng, sl, page_size, shuffle, shared_prefix // page_size)
     S = page_size
     caches = {}
     if variant == "gqa":
@@ -180,7 +191,7 @@ def make_inputs(variant: str, *, B: int, L: int, h_q: int, h_kv: int, d: int, d_
     return DecodeInputs(variant=variant, B=B, L=L, h_q=h_q, h_kv=h_kv, d=d, d_r=d_r,
                         page_size=S, num_pages=num_pages, max_pages=max_pages, scale=float(scale),
                         seqlens=sl, block_table=table, q=q, caches=caches, poison_page=poison,
-                        name=name)
+                        name=name, shared_prefix=shared_prefix)
 
 
 # Named decode workloads (shapes from the paper's decode settings).
@@ -196,10 +207,14 @@ WORKLOADS = {
                 seqlens=("uniform", 4096, 32768), scale=1.0 / math.sqrt(192), latent_scale=0.1),
     "gla2": dict(variant="gla", B=128, h_q=128, h_kv=2, d=256, d_r=64, page_size=64,
                  seqlens=("lognormal", 8192, 1.0, 65536), scale=1.0 / math.sqrt(192)),
+    # GTA shape with a 4096-token prefix shared by the batch (stored once) and per-sequence
+    # continuations of U[64, 2048] tokens: the shared-prefix decode workload
+    "gta_prefix": dict(variant="gta", B=32, h_q=32, h_kv=8, d=128, d_r=64, page_size=64,
+                       seqlens=("uniform", 64, 2048), shared_prefix=4096, scale=1.0 / math.sqrt(128)),
 }
 
 # Query lengths each workload is run at.
-WORKLOAD_QLENS = {"gta_tiny": (1,), "gta": (1,), "gqa": (1,), "mla": (1, 2), "gla2": (1, 2, 4)}
+WORKLOAD_QLENS = {"gta_tiny": (1,), "gta": (1,), "gqa": (1,), "mla": (1, 2), "gla2": (1, 2, 4), "gta_prefix": (1,)}
 
 
 def make_workload(name: str, L: int = 1, seed: int | None = None, **overrides) -> DecodeInputs:
