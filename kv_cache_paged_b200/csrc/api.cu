@@ -241,7 +241,7 @@ constexpr size_t SMEM_PER_BLOCK = 232448;
 constexpr size_t LATENT_STATIC_SMEM = 4096;
 
 struct LatentPlan {
-    bool spread;
+    bool spread, gather;
     LatentShape shape;
     bool pair;
     int n_rt, n_vc, n_sub, parts, nstage, rb;
@@ -261,7 +261,8 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
     if (p->d_r != 64) return KVD_ERR_UNSUPPORTED_SHAPE;
     LatentShape sh = latent_shape(p->d_c);
     if (sh.tok == 0) return KVD_ERR_UNSUPPORTED_SHAPE;
-    if (p->page_size % sh.tok) return KVD_ERR_UNSUPPORTED_SHAPE;
+    // pages that do not hold whole tiles are gathered token by token
+    lp->gather = p->page_size % sh.tok != 0;
     const int g = p->h_q / p->h_c;
     if (!(128 % g == 0 || g % 128 == 0)) return KVD_ERR_UNSUPPORTED_SHAPE;
     const long long R = (long long)g * p->L;
@@ -315,17 +316,24 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
         cuuint32_t box[3] = {64, (cuuint32_t)lp.rb, 1};
         if (!encode(&qm, p->q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
     }
-    {
-        cuuint64_t dims[3] = {64, tokens, (cuuint64_t)p->h_c * p->d_c / 64};
-        cuuint64_t strides[2] = {(cuuint64_t)p->h_c * p->d_c * 2, 128};
-        cuuint32_t box[3] = {64, (cuuint32_t)lp.shape.tok, (cuuint32_t)(p->d_c / 64)};
-        if (!encode(&lm, p->latent_cache, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
-    }
-    {
-        cuuint64_t dims[2] = {64, tokens};
-        cuuint64_t strides[1] = {128};
-        cuuint32_t box[2] = {64, (cuuint32_t)lp.shape.tok};
-        if (!encode(&rm, p->rope_cache, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+    if (lp.gather) {
+        memset(&lm, 0, sizeof(lm));  // gathered tiles are copied with cp.async: no cache maps
+        memset(&rm, 0, sizeof(rm));
+    } else {
+        {
+            cuuint64_t dims[3] = {64, tokens, (cuuint64_t)p->h_c * p->d_c / 64};
+            cuuint64_t strides[2] = {(cuuint64_t)p->h_c * p->d_c * 2, 128};
+            cuuint32_t box[3] = {64, (cuuint32_t)lp.shape.tok, (cuuint32_t)(p->d_c / 64)};
+            if (!encode(&lm, p->latent_cache, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                return KVD_ERR_CUDA;
+        }
+        {
+            cuuint64_t dims[2] = {64, tokens};
+            cuuint64_t strides[1] = {128};
+            cuuint32_t box[2] = {64, (cuuint32_t)lp.shape.tok};
+            if (!encode(&rm, p->rope_cache, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                return KVD_ERR_CUDA;
+        }
     }
     const size_t slots = (size_t)p->B + lp.parts - 1;
     const size_t rows = (size_t)p->L * p->h_q;
@@ -349,6 +357,9 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     a.n_sub = lp.n_sub;
     a.n_rt = lp.n_rt;
     a.row_spread = lp.spread ? 1 : 0;
+    a.gather = lp.gather ? 1 : 0;
+    a.cache0 = p->latent_cache;
+    a.cache1 = p->rope_cache;
     a.parts = lp.parts;
     a.nstage = lp.nstage;
     a.scale_log2 = p->scale * 1.4426950408889634f;
@@ -363,14 +374,18 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
             cuuint32_t box[3] = {32, (cuuint32_t)lp.rb, 1};
             if (!encode(&qrm, p->q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B)) return KVD_ERR_CUDA;
         }
-        {   // four 64-wide latent chunks (one CTA's half of a latent head) per box
+        if (lp.gather) {
+            memset(&lm2, 0, sizeof(lm2));
+            memset(&rm2, 0, sizeof(rm2));
+        }
+        if (!lp.gather) {   // four 64-wide latent chunks (one CTA's half of a latent head) per box
             cuuint64_t dims[3] = {64, tokens, (cuuint64_t)p->h_c * p->d_c / 64};
             cuuint64_t strides[2] = {(cuuint64_t)p->h_c * p->d_c * 2, 128};
             cuuint32_t box[3] = {64, (cuuint32_t)lp.shape.tok, 4};
             if (!encode(&lm2, p->latent_cache, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
                 return KVD_ERR_CUDA;
         }
-        {   // 32-wide halves of the rope rows
+        if (!lp.gather) {   // 32-wide halves of the rope rows
             cuuint64_t dims[2] = {64, tokens};
             cuuint64_t strides[1] = {128};
             cuuint32_t box[2] = {32, (cuuint32_t)lp.shape.tok};

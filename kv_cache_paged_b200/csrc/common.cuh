@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace kvd {
@@ -272,6 +273,33 @@ __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t k) { return r * 1
 __device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t k) {
     uint32_t off = r * 64u + k * 16u;
     return off ^ (((off >> 7) & 3u) << 4);
+}
+
+// Warps copy a tile, token by token, into the layout a tile box load produces: NCH 64-wide
+// chunks of the latent row (row stride lat_stride) as [chunk][tile rows][128 B] with the
+// 128-byte swizzle, chunk_bytes apart, then RW 16-byte units of the rope row as
+// [tile rows][16 RW bytes] at rope_dst (128-byte swizzle for 8 units, 64-byte for 4).  This
+// warp copies the tokens k = k0, k0 + kstep, ... (nk of them); rows[i] is the cache row of its
+// i-th token.  16-byte cp.async, consecutive lanes on consecutive bytes of a row.
+template <int NCH, int RW>
+__device__ __forceinline__ void gather_tile(uint32_t st, uint32_t chunk_bytes, const __nv_bfloat16 *lat,
+                                            size_t lat_stride, const __nv_bfloat16 *rope, size_t rope_stride,
+                                            uint32_t rope_dst, const int *rows, int k0, int kstep, int nk, int lane,
+                                            uint64_t pol) {
+    constexpr int nch = NCH, rw = RW, per_tok = NCH * 8 + RW;
+    for (int idx = lane; idx < nk * per_tok; idx += 32) {
+        const int i = idx / per_tok, u = idx - i * per_tok;
+        const int k = k0 + i * kstep;
+        const size_t row = (size_t)rows[i];
+        if (u < nch * 8) {
+            cp_async16(st + (uint32_t)(u >> 3) * chunk_bytes + sw128((uint32_t)k, (uint32_t)(u & 7)),
+                       lat + row * lat_stride + u * 8, pol);
+        } else {
+            const int v = u - nch * 8;
+            cp_async16(rope_dst + (rw == 8 ? sw128((uint32_t)k, (uint32_t)v) : sw64((uint32_t)k, (uint32_t)v)),
+                       rope + row * rope_stride + v * 8, pol);
+        }
+    }
 }
 
 // Programmatic dependent launch.

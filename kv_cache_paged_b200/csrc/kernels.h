@@ -54,6 +54,8 @@ struct LatentArgs {
     int n_sub;  // CTAs per part = h_c * row blocks * value slices
     int n_rt;   // 128-row blocks per latent head
     int row_spread;  // <= 64 rows, spread over lanes 0..15 of each TMEM lane quadrant (GLA kernel)
+    int gather;      // pages hold fewer tokens than a tile (or not a multiple): rows copied token by token
+    const void *cache0, *cache1;  // latent and rope caches (the gathered path reads them directly)
     int parts;
     int nstage;
     float scale_log2;

@@ -41,6 +41,7 @@ namespace {
 constexpr int LMAXSEG = 32;
 constexpr int DV = 256;  // value columns per CTA (fp32 accumulator columns in TMEM)
 constexpr int NSMX = 4;  // softmax warps, one per TMEM lane quadrant
+constexpr int NGATHER = 3;  // warps that copy gathered tiles (0, 2, 3)
 constexpr int LTHREADS = 32 * (4 + NSMX);  // warp 0 producer, 1 MMA, 2-3 idle, 4.. softmax
 constexpr float RESCALE_LOG2 = 8.f;
 
@@ -68,6 +69,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
     __shared__ uint32_t tmem_sh;
+    __shared__ int rows_sh[NGATHER][32];  // gathered tile: cache rows of each gather warp's tokens
 
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *q_s = smem;
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nstage; ++s) {
-            mbar_init(&full_bar[s], 1);
+            mbar_init(&full_bar[s], a.gather ? 32 * NGATHER : 1);  // gathered: one arrival per gather lane
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&qfull_bar, 1);  // q's rope chunk (TMA)
@@ -103,8 +105,10 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     if (warp == 1) tmem_alloc(&tmem_sh, 512);
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&qmap);
-        tma_prefetch_desc(&latmap);
-        tma_prefetch_desc(&ropemap);
+        if (!a.gather) {
+            tma_prefetch_desc(&latmap);
+            tma_prefetch_desc(&ropemap);
+        }
     }
     pdl_launch_dependents();
     tc_fence_before();
@@ -115,7 +119,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     // counters that persist across segment-list rounds
     uint32_t p_issued = 0, p_qloads = 0;                    // producer
     uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;        // MMA issuer
-    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0, x_q = 0;  // softmax
+    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_q = 0;  // softmax
 
     for (int skip = 0;; skip += LMAXSEG) {
         if (warp == 0) {
@@ -132,19 +136,22 @@ __global__ void __launch_bounds__(LTHREADS, 1)
         __syncthreads();
         const int nseg = nseg_sh;
 
-        if (warp == 0) {
-            // ================================================================ producer
+        if (warp == 0 || (a.gather && (warp == 2 || warp == 3))) {
+            // ================================================================ producer(s)
+            // warp 0: q's rope chunk per segment and the KV tiles; with gathered tiles warps 2
+            // and 3 copy their share of every tile too
+            const int gw = warp == 0 ? 0 : warp - 1;
             const uint64_t pol = policy_evict_first();
             bool stop = false;
             const int rb = a.row_spread ? 16 : (g < 128 ? g : 128);  // q rows per TMA box
             const int rows_tile = min(R - rt * 128, 128);          // valid rows of this row block
             for (int si = 0; si < nseg && !stop; ++si) {
                 const Seg sg = segs[si];
-                if (!mbar_wait_warp(&qempty_bar, (p_qloads & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
+                if (warp == 0 && !mbar_wait_warp(&qempty_bar, (p_qloads & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
                     stop = true;
                     break;
                 }
-                if (lane == 0) {
+                if (warp == 0 && lane == 0) {
                     mbar_arrive_expect_tx(&qfull_bar, (uint32_t)rows_tile * 128);
                     for (int run = 0; run * rb < rows_tile; ++run) {
                         const int n0 = rt * 128 + run * rb;
@@ -155,8 +162,49 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                         tma_load_3d(q_s + srow * 128, &qmap, &qfull_bar, 0, row, C::KCH - 1, pol);
                     }
                 }
-                ++p_qloads;
+                if (warp == 0) ++p_qloads;
                 const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
+                if (a.gather) {
+                    // Pages smaller than the tile (down to one token) or not a multiple of it: the
+                    // NGATHER gather warps (0, 2, 3) split the tile's tokens k = gw, gw + NGATHER, ..;
+                    // lane i resolves the cache row of the warp's i-th token (a tile ahead), then
+                    // the warp copies each token's latent and rope rows with 16-byte cp.async into
+                    // the layout the box loads produce; every lane arrives on the stage barrier
+                    // when its copies have landed.
+                    const int T = clamp_len(__ldg(a.seqlens + sg.b), max_tokens, a.L, nullptr);
+                    const __nv_bfloat16 *lat = (const __nv_bfloat16 *)a.cache0 + (size_t)c * DC;
+                    const __nv_bfloat16 *rope = (const __nv_bfloat16 *)a.cache1;
+                    const int nk = (TOK - gw + NGATHER - 1) / NGATHER;
+                    auto tok_of = [&](int t) { return min(t * TOK + gw + NGATHER * lane, T - 1); };
+                    int nxt = lane < nk ? __ldg(bt + tok_of(sg.t0) / a.page_size) : 0;
+                    for (int t = sg.t0; t < sg.t1 && !stop; ++t) {
+                        int pg = nxt;
+                        if (t + 1 < sg.t1 && lane < nk) nxt = __ldg(bt + tok_of(t + 1) / a.page_size);
+                        const uint32_t stage = p_issued % nstage;
+                        if (!mbar_wait_warp(&empty_bar[stage], ((p_issued / nstage) & 1) ^ 1, &abort_sh, a.err,
+                                            lim_ns)) {
+                            stop = true;
+                            break;
+                        }
+                        if (lane < nk) {
+                            if (pg < 0 || pg >= a.num_pages) {
+                                set_error(a.err, DEVERR_BAD_PAGE);
+                                pg = 0;
+                            }
+                            rows_sh[gw][lane] = pg * a.page_size + tok_of(t) % a.page_size;  // past T_b: repeat
+                        }
+                        __syncwarp();
+                        if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0) {
+                            const uint32_t st = smem_u32(stage_s + (size_t)stage * C::STAGE);
+                            gather_tile<DC / 64, 8>(st, C::CHUNK, lat, (size_t)a.h_c * DC, rope, 64,
+                                                    st + (DC / 64) * C::CHUNK, rows_sh[gw], gw, NGATHER, nk, lane, pol);
+                            cp_async_arrive(&full_bar[stage]);
+                        }
+                        __syncwarp();  // rows_sh is rewritten for the next tile
+                        ++p_issued;
+                    }
+                    continue;
+                }
                 const int tpp = a.page_size / TOK;
                 const int p_first = sg.t0 / tpp, p_last = (sg.t1 - 1) / tpp;
                 for (int pb = p_first; pb <= p_last && !stop; pb += 32) {
@@ -191,10 +239,15 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                 }
             }
             if (stop) {
+                // let every copy already issued land before the CTA can exit
                 volatile int never = 0;
-                const uint32_t lo = p_issued > (uint32_t)nstage ? p_issued - nstage : 0;
-                for (uint32_t k = lo; k < p_issued; ++k)
-                    mbar_wait_warp(&full_bar[k % nstage], (k / nstage) & 1, &never, nullptr, lim_ns);
+                if (a.gather) {
+                    asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's copies
+                } else {
+                    const uint32_t lo = p_issued > (uint32_t)nstage ? p_issued - nstage : 0;
+                    for (uint32_t k = lo; k < p_issued; ++k)
+                        mbar_wait_warp(&full_bar[k % nstage], (k / nstage) & 1, &never, nullptr, lim_ns);
+                }
                 if (p_qloads) mbar_wait_warp(&qfull_bar, (p_qloads - 1) & 1, &never, nullptr, lim_ns);
             }
         } else if (warp == 1) {

@@ -43,7 +43,8 @@ constexpr uint32_t P_SCOL = PDV;                          // S buffers [256, 384
 constexpr uint32_t P_QCOL = PDV + P_NSB * PTOK;           // q latent half [384, 512), bf16 pairs
 constexpr int P_NSMX = 4;                                 // softmax warps, one thread per row
 constexpr int W_PROD = 4 + P_NSMX, W_MMA = 5 + P_NSMX;
-constexpr int P_THREADS = 32 * (6 + P_NSMX);
+constexpr int P_NGATHER = 3;  // warps that copy gathered tiles: the producer and the last two
+constexpr int P_THREADS = 32 * (6 + P_NSMX + P_NGATHER - 1);
 constexpr float P_RESCALE_LOG2 = 8.f;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
@@ -59,6 +60,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
     __shared__ uint32_t tmem_sh;
+    __shared__ int rows_sh[P_NGATHER][32];  // gathered tile: cache rows of each gather warp's tokens
 
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *q_s = smem;
@@ -81,7 +83,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nstage; ++s) {
-            mbar_init(&full_bar[s], 1);
+            mbar_init(&full_bar[s], a.gather ? 32 * P_NGATHER : 1);  // gathered: one arrival per gather lane
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&qfull_bar, 1);   // q rope half (TMA)
@@ -109,8 +111,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     if (warp == W_MMA) tmem_alloc(&tmem_sh, 512);
     if (warp == W_PROD && lane == 0) {
         tma_prefetch_desc(&qrmap);
-        tma_prefetch_desc(&latmap);
-        tma_prefetch_desc(&ropemap);
+        if (!a.gather) {
+            tma_prefetch_desc(&latmap);
+            tma_prefetch_desc(&ropemap);
+        }
     }
     pdl_launch_dependents();
     tc_fence_before();
@@ -138,19 +142,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
         __syncthreads();
         const int nseg = nseg_sh;
 
-        if (warp == W_PROD) {
-            // ================================================================ producer
+        if (warp == W_PROD || (a.gather && warp > W_MMA)) {
+            // ================================================================ producer(s)
+            // W_PROD: q's rope half per segment and the KV tiles; with gathered tiles the warps
+            // after W_MMA copy their share of every tile too
+            const int gw = warp == W_PROD ? 0 : warp - W_MMA;
             const uint64_t pol = policy_evict_first();
             bool stop = false;
             const int rb = g < 128 ? g : 128;
             const int rows_tile = min(R - rt * 128, 128);
             for (int si = 0; si < nseg && !stop; ++si) {
                 const Seg sg = segs[si];
-                if (!mbar_wait_warp(&qempty_bar, (p_qloads & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
+                if (warp == W_PROD && !mbar_wait_warp(&qempty_bar, (p_qloads & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
                     stop = true;
                     break;
                 }
-                if (lane == 0) {
+                if (warp == W_PROD && lane == 0) {
                     mbar_arrive_expect_tx(&qfull_bar, (uint32_t)rows_tile * 64);
                     for (int run = 0; run * rb < rows_tile; ++run) {
                         const int n0 = rt * 128 + run * rb;
@@ -159,8 +166,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
                         tma_load_3d(q_s + run * rb * 64, &qrmap, &qfull_bar, 0, row, 16 + kr, pol);
                     }
                 }
-                ++p_qloads;
+                if (warp == W_PROD) ++p_qloads;
                 const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
+                if (a.gather) {
+                    // Pages smaller than the tile or not a multiple of it: as the GLA kernel's
+                    // gather (P_NGATHER warps split the tile's tokens), but only this CTA's latent
+                    // half (dims 256 kr ..) and rope half (dims 32 kr .., 64-byte rows).
+                    const int T = clamp_len(__ldg(a.seqlens + sg.b), max_tokens, a.L, nullptr);
+                    const __nv_bfloat16 *lat = (const __nv_bfloat16 *)a.cache0 + (size_t)c * 512 + kr * PDV;
+                    const __nv_bfloat16 *rope = (const __nv_bfloat16 *)a.cache1 + kr * 32;
+                    const int nk = (PTOK - gw + P_NGATHER - 1) / P_NGATHER;
+                    auto tok_of = [&](int t) { return min(t * PTOK + gw + P_NGATHER * lane, T - 1); };
+                    int nxt = lane < nk ? __ldg(bt + tok_of(sg.t0) / a.page_size) : 0;
+                    for (int t = sg.t0; t < sg.t1 && !stop; ++t) {
+                        int pg = nxt;
+                        if (t + 1 < sg.t1 && lane < nk) nxt = __ldg(bt + tok_of(t + 1) / a.page_size);
+                        const uint32_t stage = p_issued % nstage;
+                        if (!mbar_wait_warp(&empty_bar[stage], ((p_issued / nstage) & 1) ^ 1, &abort_sh, a.err,
+                                            lim_ns)) {
+                            stop = true;
+                            break;
+                        }
+                        if (lane < nk) {
+                            if (pg < 0 || pg >= a.num_pages) {
+                                set_error(a.err, DEVERR_BAD_PAGE);
+                                pg = 0;
+                            }
+                            rows_sh[gw][lane] = pg * a.page_size + tok_of(t) % a.page_size;  // past T_b: repeat
+                        }
+                        __syncwarp();
+                        if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0) {
+                            const uint32_t st = smem_u32(stage_s + (size_t)stage * P_STAGE);
+                            gather_tile<4, 4>(st, P_CHUNK, lat, (size_t)a.h_c * 512, rope, 64, st + 4 * P_CHUNK,
+                                              rows_sh[gw], gw, P_NGATHER, nk, lane, pol);
+                            cp_async_arrive(&full_bar[stage]);
+                        }
+                        __syncwarp();  // rows_sh is rewritten for the next tile
+                        ++p_issued;
+                    }
+                    continue;
+                }
                 const int tpp = a.page_size / PTOK;
                 const int p_first = sg.t0 / tpp, p_last = (sg.t1 - 1) / tpp;
                 for (int pb = p_first; pb <= p_last && !stop; pb += 32) {
@@ -195,10 +240,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
                 }
             }
             if (stop) {
+                // let every copy already issued land before the CTA can exit
                 volatile int never = 0;
-                const uint32_t lo = p_issued > (uint32_t)nstage ? p_issued - nstage : 0;
-                for (uint32_t k = lo; k < p_issued; ++k)
-                    mbar_wait_warp(&full_bar[k % nstage], (k / nstage) & 1, &never, nullptr, lim_ns);
+                if (a.gather) {
+                    asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's copies
+                } else {
+                    const uint32_t lo = p_issued > (uint32_t)nstage ? p_issued - nstage : 0;
+                    for (uint32_t k = lo; k < p_issued; ++k)
+                        mbar_wait_warp(&full_bar[k % nstage], (k / nstage) & 1, &never, nullptr, lim_ns);
+                }
                 if (p_qloads) mbar_wait_warp(&qfull_bar, (p_qloads - 1) & 1, &never, nullptr, lim_ns);
             }
         } else if (warp == W_MMA) {

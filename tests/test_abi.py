@@ -162,13 +162,18 @@ def _gla_params(**kw):
     (dict(h_q=127), -1),
     (dict(d_c=384), -2),                # latent width outside the compiled set
     (dict(d_r=32), -2),
-    (dict(page_size=48), -2),           # not a multiple of the 64-token tile (d_c 256)
     (dict(h_q=96, h_c=1), -2),          # 96 heads per latent head: neither divides nor is a multiple of 128
 ])
 def test_gla_validation_errors(lib, kw, expect):
     p = _gla_params(**kw)
     assert lib.kvd_gla_workspace_size(ctypes.byref(p)) == 0
     assert lib.kvd_gla_decode(ctypes.byref(p), ctypes.c_void_p(256), 1 << 30, None) == expect
+
+
+@pytest.mark.parametrize("S,d_c,h_c", [(1, 256, 2), (48, 256, 2), (1, 512, 1), (100, 512, 1)])
+def test_gla_any_page_size_is_accepted(lib, S, d_c, h_c):
+    """Pages that do not hold whole 64-token tiles are gathered token by token, not rejected."""
+    assert lib.kvd_gla_workspace_size(ctypes.byref(_gla_params(page_size=S, d_c=d_c, h_c=h_c))) > 0
 
 
 def test_gla_workspace_size(lib):

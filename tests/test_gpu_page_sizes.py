@@ -77,3 +77,41 @@ def test_page_permutation_bit_identical_at_page_size_one(cuda_device):
 def test_page_size_one_full_gta_workload(cuda_device):
     """The GTA decode workload (B 32, contexts U[1024, 8192]) with one token per page."""
     check(wl.make_workload("gta", page_size=1), what="gta workload S=1")
+
+
+def small_latent(h_c, d_c, S, **kw):
+    base = dict(B=4, L=1, h_q=128, h_kv=h_c, d=d_c, d_r=64, page_size=S, seqlens=("uniform", 1, 300), seed=S + d_c,
+                scale=0.07, latent_scale=0.1)
+    base.update(kw)
+    return wl.make_inputs("gla", **base)
+
+
+@pytest.mark.parametrize("h_c,d_c", [(2, 256), (1, 512)])
+@pytest.mark.parametrize("S", [1, 8, 16, 24, 100])
+def test_latent_small_and_ragged_page_sizes(cuda_device, h_c, d_c, S):
+    check(small_latent(h_c, d_c, S), what=f"h_c={h_c} d_c={d_c} S={S}")
+
+
+@pytest.mark.parametrize("h_c,d_c", [(2, 256), (1, 512)])
+@pytest.mark.parametrize("L,num_parts", [(2, 0), (1, 7)])
+def test_latent_page_size_one_q_len_and_splits(cuda_device, h_c, d_c, L, num_parts):
+    inp = small_latent(h_c, d_c, 1, L=L, seqlens=("uniform", L, 400), seed=50 + L)
+    check(inp, num_parts=num_parts, what=f"h_c={h_c} S=1 L={L} parts={num_parts}")
+
+
+@pytest.mark.parametrize("h_c,d_c", [(2, 256), (1, 512)])
+def test_latent_page_permutation_bit_identical_at_page_size_one(cuda_device, h_c, d_c):
+    import torch
+    inp = small_latent(h_c, d_c, 1, seed=46)
+    out1, lse1 = gu.run_gpu(inp)
+    rng = np.random.default_rng(2)
+    perm = rng.permutation(inp.num_pages)
+    inv = np.argsort(perm)
+    for k in inp.caches:
+        inp.caches[k] = np.ascontiguousarray(inp.caches[k][inv])
+    bt = inp.block_table.copy()
+    bt[bt >= 0] = perm[bt[bt >= 0]]
+    inp.block_table = bt
+    out2, lse2 = gu.run_gpu(inp)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(lse1, lse2)
