@@ -560,10 +560,18 @@ def main():
             "clocks": clocks}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        # a bounded sample of about cpu_budget seconds: a prefix of the batch, repeated when
+        # the whole step takes the oracle much less than the budget
         dt, frac, threads, n = oracle_sample(inp, args.cpu_budget)
-        line["cpu_baseline"] = {"value": dt / frac * 1e6, "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": f"first {n} of {inp.B} sequences ({frac:.3f} of the step's work) "
-                                          f"in {dt:.1f} s, scaled to the whole step"}
+        reps, total = 1, dt
+        while total < 0.5 * args.cpu_budget and reps < 1000:
+            d2, _, _, _ = oracle_sample(inp, args.cpu_budget)
+            total += d2
+            reps += 1
+        line["cpu_baseline"] = {"value": total / reps / frac * 1e6, "unit": UNIT, "cores": threads,
+                                "kind": "oracle",
+                                "sample": f"first {n} of {inp.B} sequences ({frac:.3f} of the step's work), "
+                                          f"{reps} run(s) in {total:.1f} s, mean scaled to the whole step"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:
