@@ -377,10 +377,12 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="kvd", choices=["kvd", "reference"])
-    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny", "gta_prefix"] + list(APPEND_SHAPES))
+    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny", "gta_prefix", "gta_prefix_long"] + list(APPEND_SHAPES))
     ap.add_argument("--tokens", type=int, default=65536, help="new tokens per call (append workloads)")
     ap.add_argument("--qlen", type=int, default=1)
     ap.add_argument("--page-size", type=int, default=0, help="override the workload's page size (tokens per page)")
+    ap.add_argument("--cascade", action="store_true",
+                    help="gta_prefix: batched shared-prefix decode + continuation decode + merge per step")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
@@ -457,6 +459,33 @@ def main():
     def step(qq, btt, sll):
         fn(qq, c0, c1, btt, sll, inp.scale, out=out, lse=lse, workspace=ws, stream=stream)
 
+    if args.cascade:
+        # cascade decoding of a batch-shared prefix: the prefix once for all rows of a KV group
+        # (kvd_gta_prefix_decode), each sequence's own tokens (kvd_gta_decode over its own
+        # pages), then kvd_merge_states.  The block table and seqlens a step uploads are the
+        # continuation's; the prefix's pages are cached state like the KV cache.
+        if inp.variant != "gta" or not getattr(inp, "shared_prefix", 0):
+            raise SystemExit("--cascade needs a GTA workload with a shared prefix (gta_prefix)")
+        P = inp.shared_prefix
+        pp = P // inp.page_size
+        suf = np.full_like(inp.block_table, -1)
+        suf[:, : inp.max_pages - pp] = inp.block_table[:, pp:]
+        bt_h = torch.from_numpy(suf).pin_memory()
+        sl_h = torch.from_numpy((inp.seqlens - P).astype(np.int32)).pin_memory()
+        bt, sl = bt_h.to(dev), sl_h.to(dev)
+        pre_bt = torch.from_numpy(np.ascontiguousarray(inp.block_table[:1, :pp])).to(dev)
+        pre_len = torch.tensor([P], dtype=torch.int32, device=dev)
+        out_p, lse_p = torch.empty_like(out), torch.empty_like(lse)
+        out_s, lse_s = torch.empty_like(out), torch.empty_like(lse)
+        ws_p = torch.zeros(1 << 28, dtype=torch.uint8, device=dev)
+        launches_per_step = 5  # prefix kernel + combine, continuation kernel + combine, merge
+
+        def step(qq, btt, sll):
+            binding.gta_prefix_decode(qq, c0, c1, pre_bt, pre_len, inp.scale, out=out_p, lse=lse_p, workspace=ws_p,
+                                      stream=stream)
+            binding.gta_decode(qq, c0, c1, btt, sll, inp.scale, out=out_s, lse=lse_s, workspace=ws, stream=stream)
+            binding.merge_states(out_p, lse_p, out_s, lse_s, out=out, lse=lse, stream=stream)
+
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             evict_l2()
@@ -501,6 +530,8 @@ def main():
     sampler.mark_off()
     binding.profile_events(None, None)
     kern_ms = [kev[k][0].elapsed_time(kev[k][1]) for k in range(K)]
+    if args.cascade:
+        kern_ms = step_ms  # several decode launches per step: the roofline takes the whole step
     clocks = sampler.stop()
 
     # end to end through the public API with host buffers: H2D of the step's inputs
@@ -556,7 +587,8 @@ def main():
                     "h2d_bytes_per_step": int(q.numel() * 2 + sl.numel() * 4 + bt.numel() * 4),
                     "d2h_bytes_per_step": int(out.numel() * 2 + lse.numel() * 4)},
             "gpu_launches": K * launches_per_step, "timed_region_wall_s": t_wall,
-            "kernel_timing": "second pass of K steps with events around the decode kernel",
+            "kernel_timing": ("whole steps (cascade: several decode launches per step)" if args.cascade else
+                              "second pass of K steps with events around the decode kernel"),
             "clocks": clocks}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -172,6 +172,25 @@ int kvd_gla_decode(const kvd_gla_params *p, void *workspace, size_t workspace_by
 int kvd_gta_decode_noalloc(const kvd_gta_params *p, kvd_stream_t stream);
 
 /*
+ * Shared-prefix attention (GTA) for cascade decoding: every one of the B x L query rows
+ * attends every token of ONE prefix that the whole batch shares, with no causal mask (the
+ * prefix precedes all queries).  The prefix is read once per KV group for the whole batch:
+ * the q rows of all sequences that share a group form one tensor-core tile (Hydragen-style
+ * batching of a shared prefix; the pages' shared-prefix decoding).
+ *   p->q            bf16 [B, L, h_q, d_h] as in kvd_gta_decode (q_rope already rotated)
+ *   p->tied_cache, p->rope_cache, p->page_size, p->num_pages: as in kvd_gta_decode
+ *   p->block_table  int32 [1, max_pages]: the prefix's pages
+ *   p->seqlens      int32 [1]: the prefix length T_p (T_p = 0: out = 0, lse = -inf)
+ *   p->out, p->lse  as in kvd_gta_decode: the state of each row over the prefix alone
+ * Requires d_h = 128, d_r = 64 and (h_q / h_kv) * B * L <= 8192.  The continuation (each
+ * sequence's own tokens) is decoded by kvd_gta_decode on its own pages; kvd_merge_states then
+ * gives attention over prefix + continuation.  Workspace as for kvd_gta_decode, sized by
+ * kvd_gta_prefix_workspace_size.
+ */
+size_t kvd_gta_prefix_workspace_size(const kvd_gta_params *p);
+int kvd_gta_prefix_decode(const kvd_gta_params *p, void *workspace, size_t ws_bytes, kvd_stream_t stream);
+
+/*
  * Merge two attention states of the same query rows over disjoint key sets, e.g. a prefix
  * shared by the whole batch and each sequence's own continuation (cascade decoding; the
  * combine step of "Hardware-Efficient Attention for Fast Decoding", section 3.3.2, applied

@@ -115,6 +115,10 @@ def lib():
                 f = getattr(L, f"kvd_{name}_append")
                 f.restype = ctypes.c_int
                 f.argtypes = [ctypes.POINTER(P), _vp]
+            L.kvd_gta_prefix_decode.restype = ctypes.c_int
+            L.kvd_gta_prefix_decode.argtypes = [ctypes.POINTER(GTAParams), _vp, ctypes.c_size_t, _vp]
+            L.kvd_gta_prefix_workspace_size.restype = ctypes.c_size_t
+            L.kvd_gta_prefix_workspace_size.argtypes = [ctypes.POINTER(GTAParams)]
             L.kvd_merge_states.restype = ctypes.c_int
             L.kvd_merge_states.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp]
             L.kvd_rope_q.restype = ctypes.c_int
@@ -389,4 +393,30 @@ def merge_states(out_a, lse_a, out_b, lse_b, *, out=None, lse=None, stream=None)
                                 _dev(out, "out", torch.bfloat16), _dev(lse, "lse", torch.float32), rows, d_v,
                                 _stream_ptr(stream))
     _check("kvd_merge_states", st)
+    return out, lse
+
+
+def gta_prefix_decode(q, tied_cache, rope_cache, prefix_block_table, prefix_len, scale, *, num_parts=0, out=None,
+                      lse=None, workspace=None, stream=None):
+    """Attention of every row of q [B, L, h_q, d_h] over one shared prefix (no causal mask).
+    prefix_block_table: int32 [1, max_pages] (or [max_pages]); prefix_len: int32 [1] (device)."""
+    torch = _torch()
+    B, L, h_q, d_h = q.shape
+    P, S, h_kv, _ = tied_cache.shape
+    bt = prefix_block_table.reshape(1, -1)
+    out, lse = _outputs(B, L, h_q, d_h, q.device, out, lse)
+    params = GTAParams(_dev(q, "q", torch.bfloat16, 4), _dev(tied_cache, "tied_cache", torch.bfloat16, 4),
+                       _dev(rope_cache, "rope_cache", torch.bfloat16, 3), _dev(bt, "block_table", torch.int32, 2),
+                       _dev(prefix_len, "prefix_len", torch.int32, 1), _dev(out, "out", torch.bfloat16, 4),
+                       _dev(lse, "lse", torch.float32, 3), B, L, h_q, h_kv, d_h, rope_cache.shape[-1], S, P,
+                       bt.shape[1], scale, num_parts)
+    Lb = lib()
+    size = Lb.kvd_gta_prefix_workspace_size(ctypes.byref(params))
+    if size == 0:
+        _check("kvd_gta_prefix_decode", Lb.kvd_gta_prefix_decode(ctypes.byref(params), None, 0, None))
+    if workspace is None:
+        workspace = globals()["workspace"](size, q.device)
+    st = Lb.kvd_gta_prefix_decode(ctypes.byref(params), ctypes.c_void_p(workspace.data_ptr()),
+                                  workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    _check("kvd_gta_prefix_decode", st)
     return out, lse

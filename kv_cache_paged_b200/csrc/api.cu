@@ -357,6 +357,7 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     a.n_sub = lp.n_sub;
     a.n_rt = lp.n_rt;
     a.row_spread = lp.spread ? 1 : 0;
+    a.noncausal = 0;
     a.gather = lp.gather ? 1 : 0;
     a.cache0 = p->latent_cache;
     a.cache1 = p->rope_cache;
@@ -463,6 +464,147 @@ int kvd_gta_decode(const kvd_gta_params *p, void *ws, size_t ws_bytes, kvd_strea
     return run_group(true, p->q, p->tied_cache, p->rope_cache, p->block_table, p->seqlens, p->out, p->lse, p->B,
                      p->L, p->h_q, p->h_kv, p->d_h, p->d_r, p->page_size, p->num_pages, p->max_pages, p->scale,
                      p->num_parts, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+// ----------------------------------------------------------------------------- GTA prefix
+// All B x L query rows attend one shared prefix (no causal mask) on the latent kernel: one
+// pseudo-sequence whose q positions are the batch's rows, state = a tied group (key: its first
+// 64 dims and the rope slice; value: all 128 dims).
+struct PrefixPlan {
+    LatentShape shape;
+    bool gather;
+    int n_rt, n_sub, parts, nstage, rb, rows_pos;
+    size_t smem, ws_bytes;
+};
+
+int plan_prefix(const kvd_gta_params *p, PrefixPlan *pp) {
+    if (p->B < 0 || p->L < 1 || p->h_q < 1 || p->h_kv < 1 || p->page_size < 1 || p->num_pages < 1 ||
+        p->max_pages < 1 || p->num_parts < 0)
+        return KVD_ERR_INVALID_ARG;
+    if (!std::isfinite(p->scale) || p->h_q % p->h_kv) return KVD_ERR_INVALID_ARG;
+    if (!p->q || !p->tied_cache || !p->rope_cache || !p->block_table || !p->seqlens || !p->out || !p->lse)
+        return KVD_ERR_INVALID_ARG;
+    if (!aligned(p->q, 16) || !aligned(p->tied_cache, 16) || !aligned(p->rope_cache, 16) || !aligned(p->out, 16) ||
+        !aligned(p->lse, 4) || !aligned(p->block_table, 4) || !aligned(p->seqlens, 4))
+        return KVD_ERR_INVALID_ARG;
+    if (p->d_h != 128 || p->d_r != 64) return KVD_ERR_UNSUPPORTED_SHAPE;
+    const int g = p->h_q / p->h_kv;
+    if (!(128 % g == 0 || g % 128 == 0)) return KVD_ERR_UNSUPPORTED_SHAPE;
+    const long long rows_pos = (long long)p->B * p->L;  // query positions of the pseudo-sequence
+    const long long R = (long long)g * rows_pos;
+    if ((long long)p->num_pages * p->page_size >= (1ll << 31) || (long long)p->max_pages * p->page_size >= (1ll << 31) ||
+        rows_pos * p->h_q >= (1ll << 31) || R > 128 * 64)
+        return KVD_ERR_UNSUPPORTED_SHAPE;
+    pp->shape = tied_prefix_shape();
+    pp->gather = p->page_size % pp->shape.tok != 0;
+    pp->rows_pos = (int)rows_pos;
+    pp->n_rt = (int)((R + 127) / 128);
+    pp->n_sub = p->h_kv * pp->n_rt;
+    pp->rb = g < 128 ? g : 128;
+    const size_t fixed = SMEM_PER_BLOCK - LATENT_STATIC_SMEM - 1024 - pp->shape.q_bytes;
+    int nstage = (int)(fixed / pp->shape.stage_bytes);
+    if (nstage > MAX_STAGES) nstage = MAX_STAGES;
+    if (nstage < 2) return KVD_ERR_UNSUPPORTED_SHAPE;
+    pp->nstage = nstage;
+    pp->smem = 1024 + pp->shape.q_bytes + (size_t)nstage * pp->shape.stage_bytes;
+    int parts = p->num_parts;
+    if (parts == 0) {
+        const int sms = num_sms_current();
+        if (sms <= 0) return KVD_ERR_CUDA;
+        parts = sms / pp->n_sub > 0 ? sms / pp->n_sub : 1;
+    }
+    pp->parts = parts;
+    const size_t slots = (size_t)parts;  // one pseudo-sequence: slot = part
+    const size_t rows = (size_t)rows_pos * p->h_q;
+    pp->ws_bytes = WS_HEADER + round_up(slots * rows * 4, 256) + slots * rows * 128 * 4;
+    return KVD_OK;
+}
+
+size_t kvd_gta_prefix_workspace_size(const kvd_gta_params *p) {
+    PrefixPlan pp;
+    return (p && plan_prefix(p, &pp) == KVD_OK) ? pp.ws_bytes : 0;
+}
+
+int kvd_gta_prefix_decode(const kvd_gta_params *p, void *ws, size_t ws_bytes, kvd_stream_t stream) {
+    if (!p) return KVD_ERR_INVALID_ARG;
+    PrefixPlan pp;
+    int rc = plan_prefix(p, &pp);
+    if (rc != KVD_OK) return rc;
+    if (!ws || !aligned(ws, 256)) return KVD_ERR_INVALID_ARG;
+    if (ws_bytes < pp.ws_bytes) return KVD_ERR_WORKSPACE_TOO_SMALL;
+    if (p->B == 0) return KVD_OK;
+    cudaStream_t st = (cudaStream_t)stream;
+    const cuuint64_t tokens = (cuuint64_t)p->num_pages * p->page_size;
+    CUtensorMap qm, lm, rm;
+    {
+        cuuint64_t dims[3] = {64, (cuuint64_t)pp.rows_pos * p->h_q, 2};
+        cuuint64_t strides[2] = {(cuuint64_t)p->d_h * 2, 128};
+        cuuint32_t box[3] = {64, (cuuint32_t)pp.rb, 1};
+        if (!encode(&qm, p->q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+    }
+    if (pp.gather) {
+        memset(&lm, 0, sizeof(lm));
+        memset(&rm, 0, sizeof(rm));
+    } else {
+        cuuint64_t dims[3] = {64, tokens, (cuuint64_t)p->h_kv * 2};
+        cuuint64_t strides[2] = {(cuuint64_t)p->h_kv * p->d_h * 2, 128};
+        cuuint32_t box[3] = {64, (cuuint32_t)pp.shape.tok, 2};
+        if (!encode(&lm, p->tied_cache, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+        cuuint64_t rdims[2] = {64, tokens};
+        cuuint64_t rstrides[1] = {128};
+        cuuint32_t rbox[2] = {64, (cuuint32_t)pp.shape.tok};
+        if (!encode(&rm, p->rope_cache, 2, rdims, rstrides, rbox, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+    }
+    const size_t slots = (size_t)pp.parts;
+    const size_t rows = (size_t)pp.rows_pos * p->h_q;
+    uint8_t *w = (uint8_t *)ws;
+    LatentArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = (const __nv_bfloat16 *)p->q;
+    a.block_table = p->block_table;
+    a.seqlens = p->seqlens;
+    a.out = (__nv_bfloat16 *)p->out;
+    a.lse = p->lse;
+    a.err = (uint32_t *)w;
+    a.ws_lse = (float *)(w + WS_HEADER);
+    a.ws_o = (float *)(w + WS_HEADER + round_up(slots * rows * 4, 256));
+    a.B = 1;
+    a.L = pp.rows_pos;
+    a.h_q = p->h_q;
+    a.h_c = p->h_kv;
+    a.page_size = p->page_size;
+    a.num_pages = p->num_pages;
+    a.max_pages = p->max_pages;
+    a.n_sub = pp.n_sub;
+    a.n_rt = pp.n_rt;
+    a.row_spread = 0;
+    a.noncausal = 1;
+    a.gather = pp.gather ? 1 : 0;
+    a.cache0 = p->tied_cache;
+    a.cache1 = p->rope_cache;
+    a.parts = pp.parts;
+    a.nstage = pp.nstage;
+    a.scale_log2 = p->scale * 1.4426950408889634f;
+    a.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
+    a.debug_flags = g_debug_flags.load();
+    record(g_ev_before, st);
+    if (launch_tied_prefix(qm, lm, rm, a, pp.parts * pp.n_sub, pp.smem, st) != cudaSuccess) return KVD_ERR_CUDA;
+    record(g_ev_after, st);
+    CombineArgs c;
+    c.seqlens = p->seqlens;
+    c.ws_lse = a.ws_lse;
+    c.ws_o = a.ws_o;
+    c.out = (__nv_bfloat16 *)p->out;
+    c.lse = p->lse;
+    c.B = 1;
+    c.L = 1;  // the plan of a non-causal pseudo-sequence (every position sees all tokens)
+    c.tile = pp.shape.tok;
+    c.max_tokens = p->max_pages * p->page_size;
+    c.parts = pp.parts;
+    c.rows = (int)rows;
+    c.d_v = 128;
+    if (launch_combine(c, st) != cudaSuccess) return KVD_ERR_CUDA;
+    return KVD_OK;
 }
 
 int kvd_merge_states(const void *out_a, const float *lse_a, const void *out_b, const float *lse_b, void *out,

@@ -55,6 +55,7 @@ struct LatentArgs {
     int n_rt;   // 128-row blocks per latent head
     int row_spread;  // <= 64 rows, spread over lanes 0..15 of each TMEM lane quadrant (GLA kernel)
     int gather;      // pages hold fewer tokens than a tile (or not a multiple): rows copied token by token
+    int noncausal;   // every row sees all T tokens (a shared prefix attended by all query rows)
     const void *cache0, *cache1;  // latent and rope caches (the gathered path reads them directly)
     int parts;
     int nstage;
@@ -74,6 +75,12 @@ LatentShape latent_shape(int d_c);
 
 cudaError_t launch_latent_decode(int d_c, const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
                                  const LatentArgs &a, int grid, size_t smem, cudaStream_t st);
+
+// GTA prefix attention on the latent kernel (latent_decode.cu): state = one tied group
+// (d_h 128), key = its first 64 dims + the 64-wide rope, every row sees the whole prefix.
+LatentShape tied_prefix_shape();
+cudaError_t launch_tied_prefix(const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
+                               const LatentArgs &a, int grid, size_t smem, cudaStream_t st);
 
 // d_c = 512 (MLA): CTA pairs splitting the key dimension (latent_pair.cu).
 uint32_t mla_pair_fixed_smem();   // q half + the exchange buffer

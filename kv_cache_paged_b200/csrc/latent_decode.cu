@@ -39,29 +39,35 @@ namespace kvd {
 namespace {
 
 constexpr int LMAXSEG = 32;
-constexpr int DV = 256;  // value columns per CTA (fp32 accumulator columns in TMEM)
 constexpr int NSMX = 4;  // softmax warps, one per TMEM lane quadrant
 constexpr int NGATHER = 3;  // warps that copy gathered tiles (0, 2, 3)
 constexpr int LTHREADS = 32 * (4 + NSMX);  // warp 0 producer, 1 MMA, 2-3 idle, 4.. softmax
 constexpr float RESCALE_LOG2 = 8.f;
 
-template <int DC, int TOK>
+// DC: width of the stored state the value reads (GLA: one latent head, 256; the GTA prefix
+// path: one tied group, 128); KL: its 64-wide chunks that are also key dims (GLA: all four;
+// GTA: the first, the non-RoPE half of the key).  The key is those chunks plus the 64-wide rope.
+template <int DC, int TOK, int KL>
 struct LatCfg {
-    static constexpr int KCH = (DC + 64) / 64;           // 64-wide K chunks: latent, then rope
-    static constexpr int NVC = DC / DV;                   // value slices
+    static constexpr int DV = DC;                         // value columns (fp32 accumulator columns)
+    static constexpr int NV = DC / 64;                    // 64-wide chunks of the state in a stage
+    static constexpr int KCH = NV + 1;                    // stage chunks: state, then rope
+    static constexpr int NVC = 1;                         // value slices
     static constexpr uint32_t Q_BYTES = 128 * 128;        // q's rope chunk: 128 rows x 128 B
     static constexpr uint32_t CHUNK = TOK * 128;          // one 64-dim chunk of a tile
     static constexpr uint32_t STAGE = KCH * CHUNK;
     static constexpr uint32_t S_COL = DV;                 // TMEM columns of the two S buffers
-    static constexpr uint32_t Q_COL = DV + 2 * TOK;       // TMEM columns of q's latent part (bf16 pairs)
-    static_assert(DC == DV && Q_COL + DC / 2 <= 512, "q's latent part must fit in tensor memory");
+    static constexpr uint32_t Q_COL = DV + 2 * TOK;       // TMEM columns of q's key part (bf16 pairs)
+    static constexpr int DQK = KL * 64 + 64;              // q row: key part of the state, then rope
+    static_assert(KL <= NV && Q_COL + KL * 32 <= 512, "q's key part must fit in tensor memory");
 };
 
-template <int DC, int TOK>
+template <int DC, int TOK, int KL>
 __global__ void __launch_bounds__(LTHREADS, 1)
     latent_decode_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap latmap,
                          const __grid_constant__ CUtensorMap ropemap, const LatentArgs a) {
-    using C = LatCfg<DC, TOK>;
+    using C = LatCfg<DC, TOK, KL>;
+    constexpr int DV = C::DV;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ uint64_t full_bar[MAX_STAGES], empty_bar[MAX_STAGES];
     __shared__ uint64_t qfull_bar, qtm_bar, qempty_bar, sfull_bar[2], pfull_bar[2], end_bar;
@@ -124,7 +130,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     for (int skip = 0;; skip += LMAXSEG) {
         if (warp == 0) {
             int cnt = 0;
-            plan_walk(a.seqlens, a.B, TOK, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
+            plan_walk(a.seqlens, a.B, TOK, max_tokens, a.noncausal ? 1 : a.L, part, a.parts, a.err, [&](const Seg &s) {
                 if (cnt >= skip && cnt < skip + LMAXSEG) segs[cnt - skip] = s;
                 ++cnt;
             });
@@ -159,7 +165,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                         const int row = (sg.b * a.L + i) * a.h_q + c * g + h0;
                         // spread rows: run k (rows 16k ..) lands at lanes 32k .. (see the softmax)
                         const int srow = a.row_spread ? run * 32 : run * rb;
-                        tma_load_3d(q_s + srow * 128, &qmap, &qfull_bar, 0, row, C::KCH - 1, pol);
+                        tma_load_3d(q_s + srow * 128, &qmap, &qfull_bar, 0, row, KL, pol);
                     }
                 }
                 if (warp == 0) ++p_qloads;
@@ -270,7 +276,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                     // descriptors advance by (byte offset >> 4) in their low word: one add per MMA
                     const uint64_t dk0 = umma_desc(st0 + stage * C::STAGE, 16, 1024, 2);
 #pragma unroll
-                    for (int kc = 0; kc < C::KCH - 1; ++kc)  // latent chunks: q from tensor memory
+                    for (int kc = 0; kc < KL; ++kc)  // key chunks of the state: q from tensor memory
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             umma_bf16_ts(d, tmem + C::Q_COL + kc * 32 + kk * 8,
@@ -278,7 +284,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // rope chunk: q from shared memory
                         umma_bf16(d, dq0 + (uint64_t)((kk * 32) >> 4),
-                                  dk0 + (uint64_t)(((C::KCH - 1) * C::CHUNK + kk * 32) >> 4), idesc_s, 1u);
+                                  dk0 + (uint64_t)((C::NV * C::CHUNK + kk * 32) >> 4), idesc_s, 1u);
                     umma_commit(&sfull_bar[sb]);
                     ++m_s;
                     return true;
@@ -306,7 +312,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                         }
                         tc_fence_after();
                         const uint32_t stage = (m_tile + j) % nstage;
-                        const uint64_t dv0 = umma_desc(st0 + stage * C::STAGE + vc * 4 * C::CHUNK, C::CHUNK, 1024, 2);
+                        const uint64_t dv0 = umma_desc(st0 + stage * C::STAGE + vc * C::NV * C::CHUNK, C::CHUNK, 1024, 2);
                         const uint32_t pa = tmem + C::S_COL + pb * TOK;  // P(j) over S(j)
 #pragma unroll
                         for (int kk = 0; kk < TOK / 16; ++kk)
@@ -346,7 +352,9 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                 const Seg sg = segs[si];
                 const int b = sg.b;
                 const int T = clamp_len(__ldg(a.seqlens + b), max_tokens, a.L, nullptr);
-                const int lim = row_ok ? T - a.L + i_row : -1;
+                // causal: row (i, h) sees t <= T - L + i; non-causal (prefix): every row sees all T
+                const int lim = row_ok ? (a.noncausal ? T - 1 : T - a.L + i_row) : -1;
+                const int lim_all = a.noncausal ? T - 1 : T - a.L;  // visible to every row
                 {
                     // q's latent part of this segment's rows -> tensor memory (the A operand of
                     // the score product), once the previous segment's score MMAs are done with it
@@ -356,9 +364,9 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                     }
                     tc_fence_after();
                     const uint4 *src =
-                        row_ok ? (const uint4 *)(a.q + ((size_t)(b * a.L + i_row) * a.h_q + head) * (DC + 64)) : nullptr;
+                        row_ok ? (const uint4 *)(a.q + ((size_t)(b * a.L + i_row) * a.h_q + head) * C::DQK) : nullptr;
 #pragma unroll 1
-                    for (int part16 = 0; part16 < DC / 32; ++part16) {
+                    for (int part16 = 0; part16 < KL * 2; ++part16) {
                         uint32_t w[16];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
@@ -399,7 +407,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                         }
                     }
                     ++x_s;
-                    const bool full = tile * TOK + TOK - 1 <= T - a.L && row_ok;  // no column masked
+                    const bool full = tile * TOK + TOK - 1 <= lim_all && row_ok;  // no column masked
                     if (warp_live) mx = tile_max(s, full, tok0, lim, a.scale_log2);
                     float alpha = 1.f;
                     bool need = false;
@@ -439,10 +447,10 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                     const int ttok0 = tile * TOK;
                     if (ttok0 + TOK > T) {
                         const int k0 = max(T - ttok0, 0);
-                        uint8_t *v0 = stage_s + (size_t)stage * C::STAGE + (size_t)vc * 4 * C::CHUNK;
-                        const int units = (TOK - k0) * 4 * 8;  // 16-byte units: rows x 4 chunks x 8
+                        uint8_t *v0 = stage_s + (size_t)stage * C::STAGE + (size_t)vc * C::NV * C::CHUNK;
+                        const int units = (TOK - k0) * C::NV * 8;  // 16-byte units: rows x chunks x 8
                         for (int u = st_id; u < units; u += 32 * NSMX) {
-                            const int row = k0 + u / 32, ch = (u / 8) & 3, k = u & 7;
+                            const int row = k0 + u / (C::NV * 8), ch = (u / 8) % C::NV, k = u & 7;
                             *(uint4 *)(v0 + ch * C::CHUNK + row * 128 + k * 16) = make_uint4(0, 0, 0, 0);
                         }
                     }
@@ -534,10 +542,10 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int DC, int TOK>
+template <int DC, int TOK, int KL>
 cudaError_t launch_t(const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a,
                      int grid, size_t smem, cudaStream_t st) {
-    auto k = latent_decode_kernel<DC, TOK>;
+    auto k = latent_decode_kernel<DC, TOK, KL>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<grid, LTHREADS, smem, st>>>(qm, lm, rm, a);
@@ -550,8 +558,8 @@ LatentShape latent_shape(int d_c) {
     LatentShape s{};
     if (d_c == 256) {
         s.tok = 64;
-        s.q_bytes = LatCfg<256, 64>::Q_BYTES;
-        s.stage_bytes = LatCfg<256, 64>::STAGE;
+        s.q_bytes = LatCfg<256, 64, 4>::Q_BYTES;
+        s.stage_bytes = LatCfg<256, 64, 4>::STAGE;
         s.p_bytes = 0;
     } else if (d_c == 512) {  // the CTA-pair kernel of latent_pair.cu
         s.tok = 64;
@@ -564,8 +572,22 @@ LatentShape latent_shape(int d_c) {
 
 cudaError_t launch_latent_decode(int d_c, const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
                                  const LatentArgs &a, int grid, size_t smem, cudaStream_t st) {
-    if (d_c == 256) return launch_t<256, 64>(qm, lm, rm, a, grid, smem, st);
+    if (d_c == 256) return launch_t<256, 64, 4>(qm, lm, rm, a, grid, smem, st);
     return cudaErrorInvalidValue;
+}
+
+LatentShape tied_prefix_shape() {
+    LatentShape s{};
+    s.tok = 64;
+    s.q_bytes = LatCfg<128, 64, 1>::Q_BYTES;
+    s.stage_bytes = LatCfg<128, 64, 1>::STAGE;
+    s.p_bytes = 0;
+    return s;
+}
+
+cudaError_t launch_tied_prefix(const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
+                               const LatentArgs &a, int grid, size_t smem, cudaStream_t st) {
+    return launch_t<128, 64, 1>(qm, lm, rm, a, grid, smem, st);
 }
 
 }  // namespace kvd

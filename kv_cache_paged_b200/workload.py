@@ -35,7 +35,7 @@ import numpy as np
 BF16_NAN = np.uint16(0x7FC0)
 
 # Seeds per named workload.
-SEEDS = {"gta_tiny": 0, "gta": 1, "gqa": 2, "mla": 3, "gla2": 4, "gta_prefix": 5}
+SEEDS = {"gta_tiny": 0, "gta": 1, "gqa": 2, "mla": 3, "gla2": 4, "gta_prefix": 5, "gta_prefix_long": 6}
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -211,10 +211,14 @@ WORKLOADS = {
     # continuations of U[64, 2048] tokens: the shared-prefix decode workload
     "gta_prefix": dict(variant="gta", B=32, h_q=32, h_kv=8, d=128, d_r=64, page_size=64,
                        seqlens=("uniform", 64, 2048), shared_prefix=4096, scale=1.0 / math.sqrt(128)),
+    # the same with a 32768-token shared prefix (71 MB of tied state and rope, read once per
+    # step by the batched prefix path, 32 times by a one-pass decode)
+    "gta_prefix_long": dict(variant="gta", B=32, h_q=32, h_kv=8, d=128, d_r=64, page_size=64,
+                            seqlens=("uniform", 64, 2048), shared_prefix=32768, scale=1.0 / math.sqrt(128)),
 }
 
 # Query lengths each workload is run at.
-WORKLOAD_QLENS = {"gta_tiny": (1,), "gta": (1,), "gqa": (1,), "mla": (1, 2), "gla2": (1, 2, 4), "gta_prefix": (1,)}
+WORKLOAD_QLENS = {"gta_tiny": (1,), "gta": (1,), "gqa": (1,), "mla": (1, 2), "gla2": (1, 2, 4), "gta_prefix": (1,), "gta_prefix_long": (1,)}
 
 
 def make_workload(name: str, L: int = 1, seed: int | None = None, **overrides) -> DecodeInputs:

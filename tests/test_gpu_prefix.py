@@ -99,3 +99,80 @@ def test_gta_prefix_workload(cuda_device):
     out, lse = gu.run_gpu(inp)
     ref_o, ref_l, _ = orc.decode_inputs(inp)
     gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, "gta_prefix")
+
+
+def _prefix_only_ref(inp, P):
+    """Oracle state of every query row over the prefix alone (no causal mask): each (b, i) row
+    becomes a one-row sequence whose block table is the prefix's pages and whose length is P."""
+    import copy
+    pp = P // inp.page_size
+    s = copy.copy(inp)
+    s.B, s.L = inp.B * inp.L, 1
+    s.q = np.ascontiguousarray(inp.q.reshape(inp.B * inp.L, 1, inp.h_q, -1))
+    s.block_table = np.ascontiguousarray(np.repeat(inp.block_table[:1, :pp], s.B, axis=0))
+    s.seqlens = np.full(s.B, P, np.int32)
+    ref_o, ref_l, _ = orc.decode_inputs(s)
+    return ref_o.reshape(inp.B, inp.L, inp.h_q, -1), ref_l.reshape(inp.B, inp.L, inp.h_q)
+
+
+def _prefix_gpu(inp, dev, P, num_parts=0):
+    import torch
+    pp = P // inp.page_size if P % inp.page_size == 0 else (P + inp.page_size - 1) // inp.page_size
+    bt = torch.from_numpy(np.ascontiguousarray(inp.block_table[:1, :pp])).cuda()
+    pl = torch.tensor([P], dtype=torch.int32, device="cuda")
+    return binding.gta_prefix_decode(dev["q"], dev["tied_cache"], dev["rope_cache"], bt, pl, inp.scale,
+                                     num_parts=num_parts)
+
+
+@pytest.mark.parametrize("L,num_parts", [(1, 0), (1, 5), (2, 0), (3, 2)])
+def test_batched_prefix_decode(cuda_device, L, num_parts):
+    P = 256
+    inp = prefix_inputs("gta", B=8, prefix=P, L=L, seed=70 + L)
+    out, lse = _prefix_gpu(inp, gu.to_dev(inp), P, num_parts)
+    ref_o, ref_l = _prefix_only_ref(inp, P)
+    gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, f"prefix-only L={L}", stress=True)
+
+
+@pytest.mark.parametrize("S,P", [(1, 77), (16, 96), (64, 64)])
+def test_batched_prefix_decode_page_sizes(cuda_device, S, P):
+    inp = prefix_inputs("gta", B=6, prefix=P, S=S, seed=80 + S)
+    out, lse = _prefix_gpu(inp, gu.to_dev(inp), P)
+    ref_o, ref_l = _prefix_only_ref(inp, P)
+    gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, f"prefix-only S={S}", stress=True)
+
+
+def test_cascade_batched_prefix_then_continuation(cuda_device):
+    import torch
+    P = 320
+    inp = prefix_inputs("gta", B=16, prefix=P, seed=90)
+    pp = P // inp.page_size
+    dev = gu.to_dev(inp)
+    o1, l1 = _prefix_gpu(inp, dev, P)
+    suf_table = np.full_like(inp.block_table, -1)
+    suf_table[:, : inp.max_pages - pp] = inp.block_table[:, pp:]
+    suf = _sub(inp, suf_table, inp.seqlens - P)
+    d_suf = dict(dev, block_table=torch.from_numpy(suf.block_table).cuda(), seqlens=torch.from_numpy(suf.seqlens).cuda())
+    o2, l2 = gu.run_gpu(suf, dev=d_suf)
+    o, l = binding.merge_states(o1, l1, o2, l2)
+    torch.cuda.synchronize()
+    ref_o, ref_l, _ = orc.decode_inputs(inp)
+    gu.assert_close(*gu.to_np(o, l), ref_o, ref_l, "batched prefix cascade", stress=True)
+
+
+def test_gta_prefix_workload_cascade(cuda_device):
+    """The shared-prefix workload through the batched prefix path + continuation + merge."""
+    import torch
+    inp = wl.make_workload("gta_prefix")
+    P = inp.shared_prefix
+    pp = P // inp.page_size
+    dev = gu.to_dev(inp)
+    o1, l1 = _prefix_gpu(inp, dev, P)
+    suf_table = np.full_like(inp.block_table, -1)
+    suf_table[:, : inp.max_pages - pp] = inp.block_table[:, pp:]
+    suf = _sub(inp, suf_table, inp.seqlens - P)
+    d_suf = dict(dev, block_table=torch.from_numpy(suf.block_table).cuda(), seqlens=torch.from_numpy(suf.seqlens).cuda())
+    o2, l2 = gu.run_gpu(suf, dev=d_suf)
+    o, l = binding.merge_states(o1, l1, o2, l2)
+    torch.cuda.synchronize()
+    ref_o, ref_l, _ = orc.decode_inputs(inp)
+    gu.assert_close(*gu.to_np(o, l), ref_o, ref_l, "gta_prefix cascade")
