@@ -40,7 +40,8 @@ FALLBACK_HBM_GBS, FALLBACK_TFLOPS = 6650.0, 1590.0
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 KERNEL_SOURCES = {"group": ["kv_cache_paged_b200/csrc/group_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"],
                   "latent": ["kv_cache_paged_b200/csrc/latent_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"],
-                  "pair": ["kv_cache_paged_b200/csrc/latent_pair.cu", "kv_cache_paged_b200/csrc/common.cuh"]}
+                  "pair": ["kv_cache_paged_b200/csrc/latent_pair.cu", "kv_cache_paged_b200/csrc/common.cuh"],
+                  "append": ["kv_cache_paged_b200/csrc/append.cu", "kv_cache_paged_b200/csrc/common.cuh"]}
 KERNEL_NAMES = {"group": "group_decode_kernel", "latent": "latent_decode_kernel", "pair": "mla_pair_kernel"}
 
 
@@ -360,7 +361,8 @@ def run_append(args, rank):
             "warmup": args.warmup, "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 copy, f64 rotation", "data": "synthetic", "config": cfg,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                         "traffic": None, "peak_source": src, "kernel": "append_kernel", "kernel_us": us},
+                         "traffic": committed_traffic("append", args.workload, 1) if n == 65536 else None,
+                         "peak_source": src, "kernel": "append_kernel", "kernel_us": us},
             "e2e": {"value": statistics.mean(e2e), "unit": "us/call", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": 2},
             "gpu_launches": args.steps, "clocks": clocks}
