@@ -585,7 +585,8 @@ def main():
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
     roof["kernel"] = KERNEL_NAMES[variant_kind]
     roof["kernel_us"] = t_kern * 1e3
-    roof["traffic"] = committed_traffic(variant_kind, args.workload, inp.L)
+    # the committed ncu traffic was taken on the workload's own page size
+    roof["traffic"] = committed_traffic(variant_kind, args.workload, inp.L) if args.page_size <= 0 else None
     roof["roofline_us"] = accounting.roofline_us(nbytes, flops, hbm, tfl)
 
     kv_gbs = aggregate(t_step * 1e3, kvb, 1)
