@@ -407,8 +407,13 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                         }
                     }
                     ++x_s;
-                    const bool full = tile * TOK + TOK - 1 <= lim_all && row_ok;  // no column masked
-                    if (warp_live) mx = tile_max(s, full, tok0, lim, a.scale_log2);
+                    // no column masked; the same for every lane of the warp (rows past R are
+                    // handled by forcing their maximum to -inf: their S is garbage, never used)
+                    const bool full = tile * TOK + TOK - 1 <= lim_all;
+                    if (warp_live) {
+                        mx = tile_max(s, full, tok0, lim, a.scale_log2);
+                        if (!row_ok) mx = -INFINITY;
+                    }
                     float alpha = 1.f;
                     bool need = false;
                     if (mx != -INFINITY) {

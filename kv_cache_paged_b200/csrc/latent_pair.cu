@@ -471,8 +471,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
                     ++x_s;
 
                     float mx = -INFINITY;
-                    const bool full = tile * PTOK + PTOK - 1 <= T - a.L && row_ok;  // no column masked
-                    if (warp_live) mx = tile_max(s, full, tok0, lim, a.scale_log2);
+                    // no column masked; the same for every lane of the warp (rows past R: -inf)
+                    const bool full = tile * PTOK + PTOK - 1 <= T - a.L;
+                    if (warp_live) {
+                        mx = tile_max(s, full, tok0, lim, a.scale_log2);
+                        if (!row_ok) mx = -INFINITY;
+                    }
                     float alpha = 1.f;
                     bool need = false;
                     if (mx != -INFINITY) {
