@@ -379,7 +379,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="kvd", choices=["kvd", "reference"])
-    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny", "gta_prefix", "gta_prefix_long"] + list(APPEND_SHAPES))
+    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny", "gta_prefix", "gta_prefix_long", "gla8"] + list(APPEND_SHAPES))
     ap.add_argument("--tokens", type=int, default=65536, help="new tokens per call (append workloads)")
     ap.add_argument("--qlen", type=int, default=1)
     ap.add_argument("--page-size", type=int, default=0, help="override the workload's page size (tokens per page)")

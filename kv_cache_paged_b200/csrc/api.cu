@@ -241,7 +241,8 @@ constexpr size_t SMEM_PER_BLOCK = 232448;
 constexpr size_t LATENT_STATIC_SMEM = 4096;
 
 struct LatentPlan {
-    bool spread, gather;
+    int spread;  // rows per lane quadrant when the rows are spread (0: not spread)
+    bool gather;
     LatentShape shape;
     bool pair;
     int n_rt, n_vc, n_sub, parts, nstage, rb;
@@ -275,10 +276,17 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
     lp->n_vc = lp->pair ? 1 : p->d_c / 256;
     lp->n_sub = p->h_c * lp->n_rt * lp->n_vc;
     const int ctas_per_sub = lp->pair ? 2 : 1;
-    // the GLA kernel spreads at most 64 rows over the four TMEM lane quadrants (16 each), which
-    // needs the q rows in 16-row runs that stay inside one query position
-    lp->spread = !lp->pair && R <= 64 && g % 16 == 0;
-    lp->rb = lp->spread ? 16 : (g < 128 ? g : 128);
+    // the GLA kernel spreads at most 64 rows evenly over the four TMEM lane quadrants
+    // (rpq = 4, 8 or 16 rows each), which needs the q rows in rpq-row runs that stay inside one
+    // query position (g % rpq == 0)
+    lp->spread = 0;
+    if (!lp->pair && R <= 64)
+        for (int rpq = 4; rpq <= 16; rpq *= 2)
+            if (4 * rpq >= R && g % rpq == 0) {
+                lp->spread = rpq;
+                break;
+            }
+    lp->rb = lp->spread ? lp->spread : (g < 128 ? g : 128);
     const size_t fixed = SMEM_PER_BLOCK - LATENT_STATIC_SMEM - 1024 - sh.q_bytes - sh.p_bytes;
     int nstage = (int)(fixed / sh.stage_bytes);
     if (nstage > MAX_STAGES) nstage = MAX_STAGES;
@@ -356,7 +364,7 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     a.max_pages = p->max_pages;
     a.n_sub = lp.n_sub;
     a.n_rt = lp.n_rt;
-    a.row_spread = lp.spread ? 1 : 0;
+    a.row_spread = lp.spread;
     a.noncausal = 0;
     a.gather = lp.gather ? 1 : 0;
     a.cache0 = p->latent_cache;

@@ -53,7 +53,7 @@ struct LatentArgs {
     int B, L, h_q, h_c, page_size, num_pages, max_pages;
     int n_sub;  // CTAs per part = h_c * row blocks * value slices
     int n_rt;   // 128-row blocks per latent head
-    int row_spread;  // <= 64 rows, spread over lanes 0..15 of each TMEM lane quadrant (GLA kernel)
+    int row_spread;  // <= 64 rows spread over the TMEM lane quadrants: rows per quadrant (0: off)
     int gather;      // pages hold fewer tokens than a tile (or not a multiple): rows copied token by token
     int noncausal;   // every row sees all T tokens (a shared prefix attended by all query rows)
     const void *cache0, *cache1;  // latent and rope caches (the gathered path reads them directly)

@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
             const int gw = warp == 0 ? 0 : warp - 1;
             const uint64_t pol = policy_evict_first();
             bool stop = false;
-            const int rb = a.row_spread ? 16 : (g < 128 ? g : 128);  // q rows per TMA box
+            const int rb = a.row_spread ? a.row_spread : (g < 128 ? g : 128);  // q rows per TMA box
             const int rows_tile = min(R - rt * 128, 128);          // valid rows of this row block
             for (int si = 0; si < nseg && !stop; ++si) {
                 const Seg sg = segs[si];
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                         const int n0 = rt * 128 + run * rb;
                         const int i = n0 / g, h0 = n0 % g;
                         const int row = (sg.b * a.L + i) * a.h_q + c * g + h0;
-                        // spread rows: run k (rows 16k ..) lands at lanes 32k .. (see the softmax)
+                        // spread rows: run k (rows k * row_spread ..) lands at lanes 32k .. (see the softmax)
                         const int srow = a.row_spread ? run * 32 : run * rb;
                         tma_load_3d(q_s + srow * 128, &qmap, &qfull_bar, 0, row, KL, pol);
                     }
@@ -329,14 +329,15 @@ __global__ void __launch_bounds__(LTHREADS, 1)
             // ================================================================ softmax / epilogue
             // Four warps, one thread per row: warp w reads TMEM lanes 32 (w % 4) .. + 31 and the
             // whole 64-token S row of its thread, so no row value crosses threads.  When a CTA has
-            // at most 64 rows (GLA-2 at q_len 1) they are spread over lanes 0..15 of every lane
-            // quadrant (row n at lane 32 (n / 16) + n % 16): each of the four warps, one per SM
-            // sub-partition, then holds 16 rows.
+            // at most 64 rows (GLA-2 at q_len 1: 64; GLA-8: 16 L) they are spread evenly over the
+            // four lane quadrants, row_spread rows each (row n at lane 32 (n / row_spread) +
+            // n % row_spread), so that each of the four warps, one per SM sub-partition, holds
+            // a quarter of them.
             const int st_id = threadIdx.x - 128;         // 0 .. 127
             const int r = (warp & 3) * 32 + lane;        // TMEM lane
             const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
             const bool spread = a.row_spread != 0;
-            const int n_row = spread ? ((lane < 16) ? (warp & 3) * 16 + lane : R) : rt * 128 + r;
+            const int n_row = spread ? ((lane < a.row_spread) ? (warp & 3) * a.row_spread + lane : R) : rt * 128 + r;
             const bool row_ok = n_row < R;
             const bool warp_live = spread || rt * 128 + (warp & 3) * 32 < R;  // some row of this warp is real
             const int i_row = row_ok ? n_row / g : 0;

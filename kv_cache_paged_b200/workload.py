@@ -35,7 +35,7 @@ import numpy as np
 BF16_NAN = np.uint16(0x7FC0)
 
 # Seeds per named workload.
-SEEDS = {"gta_tiny": 0, "gta": 1, "gqa": 2, "mla": 3, "gla2": 4, "gta_prefix": 5, "gta_prefix_long": 6}
+SEEDS = {"gta_tiny": 0, "gta": 1, "gqa": 2, "mla": 3, "gla2": 4, "gta_prefix": 5, "gta_prefix_long": 6, "gla8": 7}
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -207,6 +207,9 @@ WORKLOADS = {
                 seqlens=("uniform", 4096, 32768), scale=1.0 / math.sqrt(192), latent_scale=0.1),
     "gla2": dict(variant="gla", B=128, h_q=128, h_kv=2, d=256, d_r=64, page_size=64,
                  seqlens=("lognormal", 8192, 1.0, 65536), scale=1.0 / math.sqrt(192)),
+    # GLA-8 (NEXT-3): eight 256-wide latent heads, 16 query heads each, GLA-2's contexts
+    "gla8": dict(variant="gla", B=128, h_q=128, h_kv=8, d=256, d_r=64, page_size=64,
+                 seqlens=("lognormal", 8192, 1.0, 65536), scale=1.0 / math.sqrt(192)),
     # GTA shape with a 4096-token prefix shared by the batch (stored once) and per-sequence
     # continuations of U[64, 2048] tokens: the shared-prefix decode workload
     "gta_prefix": dict(variant="gta", B=32, h_q=32, h_kv=8, d=128, d_r=64, page_size=64,
@@ -218,7 +221,7 @@ WORKLOADS = {
 }
 
 # Query lengths each workload is run at.
-WORKLOAD_QLENS = {"gta_tiny": (1,), "gta": (1,), "gqa": (1,), "mla": (1, 2), "gla2": (1, 2, 4), "gta_prefix": (1,), "gta_prefix_long": (1,)}
+WORKLOAD_QLENS = {"gta_tiny": (1,), "gta": (1,), "gqa": (1,), "mla": (1, 2), "gla2": (1, 2, 4), "gta_prefix": (1,), "gta_prefix_long": (1,), "gla8": (1, 2, 4, 8)}
 
 
 def make_workload(name: str, L: int = 1, seed: int | None = None, **overrides) -> DecodeInputs:

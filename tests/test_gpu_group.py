@@ -222,3 +222,11 @@ def test_cuda_graph_capture_and_replay(cuda_device):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("variant", ["gqa", "gta"])
+@pytest.mark.parametrize("L", [4, 8])
+def test_longer_speculation(cuda_device, variant, L):
+    """q_len up to 8 (32 query rows per KV group): the warp-MMA kernel's largest row block."""
+    inp = small(variant, L=L, seqlens=("uniform", L, 600), seed=110 + L)
+    check(inp, num_parts=7)

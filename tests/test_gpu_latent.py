@@ -115,3 +115,11 @@ def test_gla2_workload_full_size(cuda_device, L):
     inp = wl.make_workload("gla2", L=L)
     longest = int(np.argmax(inp.seqlens))
     check(inp, b_sample=[0, 5, 40, 77, 127, longest], what=f"GLA-2 workload L={L}", stress=False)
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 8])
+def test_gla8_speculation_lengths(cuda_device, L):
+    """GLA-8 (16 query heads per latent head) at q_len 1..8: 16 L rows per latent head,
+    spread over the lane quadrants when at most 64."""
+    inp = small(8, 256, h_q=128, L=L, seqlens=("uniform", L, 400), seed=100 + L)
+    check(inp, num_parts=5, what=f"GLA-8 L={L}")
