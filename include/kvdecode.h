@@ -74,7 +74,7 @@ typedef struct CUstream_st *kvd_stream_t; /* same handle as cudaStream_t; NULL =
 enum {
     KVD_OK = 0,
     KVD_ERR_INVALID_ARG = -1,        /* null/misaligned pointer, inconsistent sizes */
-    KVD_ERR_UNSUPPORTED_SHAPE = -2,  /* head dims / page size outside the compiled set */
+    KVD_ERR_UNSUPPORTED_SHAPE = -2,  /* head dims or group size outside the compiled set */
     KVD_ERR_WORKSPACE_TOO_SMALL = -3,
     KVD_ERR_CUDA = -4,               /* a CUDA runtime call or launch failed */
     KVD_ERR_DEVICE = -5              /* kvd_read_device_error found flags set */
@@ -88,8 +88,10 @@ enum {
 };
 
 /*
- * GQA (and MQA/MHA).  d in {64, 128}; h_q % h_kv == 0; (h_q / h_kv) * L <= 32;
- * page_size a multiple of 16.
+ * GQA (and MQA/MHA).  d in {64, 128}; h_q % h_kv == 0; (h_q / h_kv) * L <= 32; any
+ * page_size >= 1: pages holding whole 16- or 32-token tiles are loaded with one tensor-map box
+ * per tile, smaller pages (down to one token) or sizes that are not a multiple of 16 are
+ * gathered token by token (slower; the same results).
  */
 typedef struct {
     const void *q;            /* bf16 [B, L, h_q, d] */
@@ -122,8 +124,9 @@ typedef struct {
 } kvd_gta_params;
 
 /*
- * GLA / MLA (absorbed).  d_c in {256, 512}, d_r == 64, h_q % h_c == 0,
- * (h_q / h_c) * L <= 256, page_size a multiple of 64.
+ * GLA / MLA (absorbed).  d_c in {256, 512}, d_r == 64, h_q % h_c == 0, h_q / h_c divides or is
+ * a multiple of 128, (h_q / h_c) * L <= 8192; any page_size >= 1 (multiples of 64 load
+ * whole tiles, other sizes are gathered token by token).
  */
 typedef struct {
     const void *q;            /* bf16 [B, L, h_q, d_c + d_r] = [latent ++ rope] */
