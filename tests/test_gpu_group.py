@@ -230,3 +230,11 @@ def test_longer_speculation(cuda_device, variant, L):
     """q_len up to 8 (32 query rows per KV group): the warp-MMA kernel's largest row block."""
     inp = small(variant, L=L, seqlens=("uniform", L, 600), seed=110 + L)
     check(inp, num_parts=7)
+
+
+@pytest.mark.parametrize("variant", ["gqa", "gta"])
+@pytest.mark.parametrize("S", [64, 1])
+def test_more_segments_than_one_plan_chunk(cuda_device, variant, S):
+    """300 short sequences on 2 parts: each CTA walks its plan in chunks of 128 segments."""
+    inp = small(variant, B=300, page_size=S, seqlens=("uniform", 1, 40), seed=120 + S)
+    check(inp, num_parts=2, what=f"{variant} 300 sequences S={S}")

@@ -123,3 +123,11 @@ def test_gla8_speculation_lengths(cuda_device, L):
     spread over the lane quadrants when at most 64."""
     inp = small(8, 256, h_q=128, L=L, seqlens=("uniform", L, 400), seed=100 + L)
     check(inp, num_parts=5, what=f"GLA-8 L={L}")
+
+
+@pytest.mark.parametrize("h_c,d_c", [(2, 256), (1, 512)])
+@pytest.mark.parametrize("S", [64, 1])
+def test_latent_more_segments_than_one_plan_chunk(cuda_device, h_c, d_c, S):
+    """80 short sequences on one part: the CTA walks its plan in chunks of 32 segments."""
+    inp = small(h_c, d_c, B=80, page_size=S, seqlens=("uniform", 1, 90), seed=130 + S + h_c)
+    check(inp, num_parts=1, what=f"h_c={h_c} 80 sequences S={S}")

@@ -176,3 +176,24 @@ def test_gta_prefix_workload_cascade(cuda_device):
     torch.cuda.synchronize()
     ref_o, ref_l, _ = orc.decode_inputs(inp)
     gu.assert_close(*gu.to_np(o, l), ref_o, ref_l, "gta_prefix cascade")
+
+
+def test_batched_prefix_more_than_128_rows(cuda_device):
+    """48 sequences x 4 heads per KV group = 192 rows: two 128-row blocks per group."""
+    P = 128
+    inp = prefix_inputs("gta", B=48, prefix=P, seed=95)
+    out, lse = _prefix_gpu(inp, gu.to_dev(inp), P)
+    ref_o, ref_l = _prefix_only_ref(inp, P)
+    gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, "prefix-only 192 rows", stress=True)
+
+
+def test_batched_prefix_empty_prefix(cuda_device):
+    import torch
+    inp = prefix_inputs("gta", B=4, prefix=64, seed=96)
+    dev = gu.to_dev(inp)
+    bt = torch.from_numpy(np.ascontiguousarray(inp.block_table[:1, :1])).cuda()
+    out, lse = binding.gta_prefix_decode(dev["q"], dev["tied_cache"], dev["rope_cache"], bt,
+                                         torch.zeros(1, dtype=torch.int32, device="cuda"), inp.scale)
+    torch.cuda.synchronize()
+    o, l = gu.to_np(out, lse)
+    assert np.all(o == 0) and np.all(np.isneginf(l))
