@@ -279,25 +279,40 @@ __device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t k) {
 // chunks of the latent row (row stride lat_stride) as [chunk][tile rows][128 B] with the
 // 128-byte swizzle, chunk_bytes apart, then RW 16-byte units of the rope row as
 // [tile rows][16 RW bytes] at rope_dst (128-byte swizzle for 8 units, 64-byte for 4).  This
-// warp copies the tokens k = k0, k0 + kstep, ... (nk of them); rows[i] is the cache row of its
-// i-th token.  16-byte cp.async, consecutive lanes on consecutive bytes of a row.
+// warp copies the tokens k = k0, k0 + kstep, ... (nk <= 32 of them); lane i holds `myrow`, the
+// cache row of its i-th token.  A 16-byte cp.async instruction moves at most 512 bytes and
+// the SM retires only so many of them per cycle, so every instruction is made full: per token
+// 512 consecutive bytes of the latent row (lane l: 16-byte unit l % 8 of chunk l / 8 + 4 j),
+// and the rope rows of 32 / RW tokens at once.  The per-lane parts of the addresses are fixed
+// for the whole call.
 template <int NCH, int RW>
 __device__ __forceinline__ void gather_tile(uint32_t st, uint32_t chunk_bytes, const __nv_bfloat16 *lat,
                                             size_t lat_stride, const __nv_bfloat16 *rope, size_t rope_stride,
-                                            uint32_t rope_dst, const int *rows, int k0, int kstep, int nk, int lane,
+                                            uint32_t rope_dst, int myrow, int k0, int kstep, int nk, int lane,
                                             uint64_t pol) {
-    constexpr int nch = NCH, rw = RW, per_tok = NCH * 8 + RW;
-    for (int idx = lane; idx < nk * per_tok; idx += 32) {
-        const int i = idx / per_tok, u = idx - i * per_tok;
-        const int k = k0 + i * kstep;
-        const size_t row = (size_t)rows[i];
-        if (u < nch * 8) {
-            cp_async16(st + (uint32_t)(u >> 3) * chunk_bytes + sw128((uint32_t)k, (uint32_t)(u & 7)),
-                       lat + row * lat_stride + u * 8, pol);
-        } else {
-            const int v = u - nch * 8;
-            cp_async16(rope_dst + (rw == 8 ? sw128((uint32_t)k, (uint32_t)v) : sw64((uint32_t)k, (uint32_t)v)),
-                       rope + row * rope_stride + v * 8, pol);
+    constexpr int UNITS = NCH * 8, NJ = (UNITS + 31) / 32, TPI = 32 / RW;
+    const uint32_t dst_l = st + (uint32_t)(lane >> 3) * chunk_bytes;
+    const uint32_t c_l = (uint32_t)(lane & 7);
+    const __nv_bfloat16 *lat_l = lat + lane * 8;
+#pragma unroll 2
+    for (int i = 0; i < nk; ++i) {
+        const uint32_t k = (uint32_t)(k0 + i * kstep);
+        const size_t row = (size_t)__shfl_sync(0xffffffffu, myrow, i);
+        const uint32_t dst = dst_l + k * 128u + ((c_l ^ (k & 7u)) << 4);
+        const __nv_bfloat16 *src = lat_l + row * lat_stride;
+#pragma unroll
+        for (int j = 0; j < NJ; ++j)
+            if (UNITS % 32 == 0 || lane + 32 * j < UNITS) cp_async16(dst + (uint32_t)(4 * j) * chunk_bytes, src + 256 * j, pol);
+    }
+    // rope: lane l copies unit l % RW of the warp's token i0 + l / RW
+    const uint32_t ru = (uint32_t)(lane % RW);
+    const __nv_bfloat16 *rope_l = rope + ru * 8;
+    for (int i0 = 0; i0 < nk; i0 += TPI) {
+        const int i = i0 + lane / RW;
+        const size_t row = (size_t)__shfl_sync(0xffffffffu, myrow, i & 31);
+        if (i < nk) {
+            const uint32_t k = (uint32_t)(k0 + i * kstep);
+            cp_async16(rope_dst + (RW == 8 ? sw128(k, ru) : sw64(k, ru)), rope_l + row * rope_stride, pol);
         }
     }
 }

@@ -132,21 +132,39 @@ __global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
                         }
                         const int myrow = page * a.page_size + tok % a.page_size;
                         if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || issued != 0) {
+                            // lane l moves 16-byte unit l % 8 of chunk l / 8 + 4 j of each token: the
+                            // per-lane parts of both addresses are fixed, a token adds its row and slot
                             const uint32_t st = smem_u32(smem + (size_t)stage * a.stage_bytes);
-                            const int per_tok = nch * 8;  // 16-byte units of a token in K / tied / V
-#pragma unroll 1
+                            const uint32_t dst_l = st + (uint32_t)((lane >> 3) * TT) * 128u;
+                            const uint32_t c_l = (uint32_t)(lane & 7);
+                            const int nj = (nch * 8 - lane + 31) / 32;  // this lane's units of a row
+#pragma unroll
                             for (int i = 0; i < TPW; ++i) {
-                                const int k = pw + GATHER_WARPS * i;
-                                const int row = __shfl_sync(0xffffffffu, myrow, i);
-                                for (int u = lane; u < per_tok; u += 32) {
-                                    const int z = u >> 3, c = u & 7;
-                                    const uint32_t so = sw128((uint32_t)(z * TT + k), (uint32_t)c);
-                                    cp_async16(st + so, c0 + (size_t)row * row_elems + u * 8, pol);
-                                    if (!TIED) cp_async16(st + kv_tile + so, c1 + (size_t)row * row_elems + u * 8, pol);
+                                const uint32_t k = (uint32_t)(pw + GATHER_WARPS * i);
+                                const size_t row = (size_t)__shfl_sync(0xffffffffu, myrow, i);
+                                const uint32_t dst = dst_l + k * 128u + ((c_l ^ (k & 7u)) << 4);
+                                const __nv_bfloat16 *s0 = c0 + row * row_elems + lane * 8;
+#pragma unroll 4
+                                for (int j = 0; j < nj; ++j) {
+                                    const uint32_t d = dst + (uint32_t)(4 * j * TT) * 128u;
+                                    cp_async16(d, s0 + 256 * j, pol);
+                                    if (!TIED) cp_async16(d + kv_tile, c1 + row * row_elems + lane * 8 + 256 * j, pol);
                                 }
-                                if (TIED && lane < RU)
-                                    cp_async16(st + kv_tile + (DR == 64 ? sw128(k, lane) : sw64(k, lane)),
-                                               c1 + (size_t)row * DR + lane * 8, pol);
+                            }
+                            if constexpr (TIED) {
+                                // rope rows, 32 / RU tokens per instruction: lane l copies unit l % RU
+                                // of token pw + GATHER_WARPS (i0 + l / RU)
+                                const uint32_t ru = (uint32_t)(lane % RU);
+#pragma unroll
+                                for (int i0 = 0; i0 < TPW; i0 += 32 / RU) {
+                                    const int i = i0 + lane / RU;
+                                    const size_t row = (size_t)__shfl_sync(0xffffffffu, myrow, i & 31);
+                                    if (i < TPW) {
+                                        const uint32_t k = (uint32_t)(pw + GATHER_WARPS * i);
+                                        cp_async16(st + kv_tile + (DR == 64 ? sw128(k, ru) : sw64(k, ru)),
+                                                   c1 + row * DR + ru * 8, pol);
+                                    }
+                                }
                             }
                             cp_async_arrive(&full_bar[stage]);
                         }

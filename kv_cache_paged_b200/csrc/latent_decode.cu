@@ -75,7 +75,6 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
     __shared__ uint32_t tmem_sh;
-    __shared__ int rows_sh[NGATHER][32];  // gathered tile: cache rows of each gather warp's tokens
 
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *q_s = smem;
@@ -192,21 +191,20 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                             stop = true;
                             break;
                         }
+                        int myrow = 0;  // cache row of this warp's lane-th token (past T_b: repeat)
                         if (lane < nk) {
                             if (pg < 0 || pg >= a.num_pages) {
                                 set_error(a.err, DEVERR_BAD_PAGE);
                                 pg = 0;
                             }
-                            rows_sh[gw][lane] = pg * a.page_size + tok_of(t) % a.page_size;  // past T_b: repeat
+                            myrow = pg * a.page_size + tok_of(t) % a.page_size;
                         }
-                        __syncwarp();
                         if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0) {
                             const uint32_t st = smem_u32(stage_s + (size_t)stage * C::STAGE);
                             gather_tile<DC / 64, 8>(st, C::CHUNK, lat, (size_t)a.h_c * DC, rope, 64,
-                                                    st + (DC / 64) * C::CHUNK, rows_sh[gw], gw, NGATHER, nk, lane, pol);
+                                                    st + (DC / 64) * C::CHUNK, myrow, gw, NGATHER, nk, lane, pol);
                             cp_async_arrive(&full_bar[stage]);
                         }
-                        __syncwarp();  // rows_sh is rewritten for the next tile
                         ++p_issued;
                     }
                     continue;

@@ -60,7 +60,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
     __shared__ uint32_t tmem_sh;
-    __shared__ int rows_sh[P_NGATHER][32];  // gathered tile: cache rows of each gather warp's tokens
 
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t *q_s = smem;
@@ -187,21 +186,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
                             stop = true;
                             break;
                         }
+                        int myrow = 0;  // cache row of this warp's lane-th token (past T_b: repeat)
                         if (lane < nk) {
                             if (pg < 0 || pg >= a.num_pages) {
                                 set_error(a.err, DEVERR_BAD_PAGE);
                                 pg = 0;
                             }
-                            rows_sh[gw][lane] = pg * a.page_size + tok_of(t) % a.page_size;  // past T_b: repeat
+                            myrow = pg * a.page_size + tok_of(t) % a.page_size;
                         }
-                        __syncwarp();
                         if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0) {
                             const uint32_t st = smem_u32(stage_s + (size_t)stage * P_STAGE);
                             gather_tile<4, 4>(st, P_CHUNK, lat, (size_t)a.h_c * 512, rope, 64, st + 4 * P_CHUNK,
-                                              rows_sh[gw], gw, P_NGATHER, nk, lane, pol);
+                                              myrow, gw, P_NGATHER, nk, lane, pol);
                             cp_async_arrive(&full_bar[stage]);
                         }
-                        __syncwarp();  // rows_sh is rewritten for the next tile
                         ++p_issued;
                     }
                     continue;
