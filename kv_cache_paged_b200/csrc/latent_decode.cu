@@ -9,26 +9,26 @@
 // (MLA: ~2 h_q FLOPs per byte, near the B200 ridge; GLA-2: ~h_q).
 //
 // One CTA owns one contiguous part of the (sequence, TOK-token tile) stream, one
-// latent head c, one 128-row block of the (q position, head) rows and one
-// 256-wide slice of the value (MLA's 512 value columns are split over two
-// neighbouring CTAs, since a 128 x 512 fp32 accumulator alone fills all of tensor
-// memory).  Roles:
-//   warp 0      producer: q rows of the segment, then per tile one 3-D TMA for
+// latent head c and one 128-row block of the (q position, head) rows (MLA's 512 value
+// columns do not fit one CTA's tensor memory next to the scores; it runs on the CTA-pair
+// kernel instead).  Roles:
+//   warp 0      producer: q's rope chunk of the segment, then per tile one 3-D TMA for
 //               the latent rows and one for the rope rows (128 B swizzle), into an
-//               n-stage mbarrier ring; block-table entries a warp at a time.
+//               n-stage mbarrier ring; block-table entries a warp at a time.  Pages that
+//               do not hold whole tiles are gathered token by token with cp.async by
+//               warps 0, 2 and 3 into the same layout.
 //   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM S buffers
-//               (M 128 rows, N TOK tokens, K d_c + d_r), then O += P V (N 256,
-//               K TOK, V read MN-major straight from the latent tile); completion
-//               reported with tcgen05.commit on mbarriers.
-//   warps 4..11 softmax: a row (TMEM lane) is shared by two threads, one per column half
-//               of the tile; each loads its half of the S row, masks, runs the fp32
-//               online softmax in base 2 with a lazy rescale (O in TMEM is
-//               rescaled only when the running max grows by more than 2^8), write
-//               P (bf16 pairs) back into tensor memory, double-buffered, where the
-//               P.V product reads it as its A operand; epilogue out / lse or split
-//               partials.
-// Tensor memory (512 columns): O [0, 256), S buffers [256, 256 + 2 TOK), P buffers
-// after them (TOK / 2 columns each).
+//               (M 128 rows, N TOK tokens, K d_c + d_r; q's latent part is the A operand
+//               from tensor memory, its rope chunk from shared memory), then O += P V
+//               (N d_c, K TOK, V read MN-major straight from the latent tile, P the A
+//               operand from tensor memory); completion reported with tcgen05.commit.
+//   warps 4..7  softmax, one thread per row (TMEM lane): load the S row, mask, fp32 online
+//               softmax in base 2 with a lazy rescale (O in TMEM is rescaled only when the
+//               running max grows by more than 2^8), write P as bf16 pairs over S in the
+//               same TMEM columns; at segment start they write q's latent part into TMEM;
+//               epilogue out / lse or split partials.
+// Tensor memory (512 columns): O [0, d_c), the two S/P buffers [d_c, d_c + 2 TOK), q's
+// key part (bf16 pairs) after them.
 #include <cuda_bf16.h>
 
 #include "common.cuh"

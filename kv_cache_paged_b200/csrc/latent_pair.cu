@@ -16,7 +16,8 @@
 // memory at the start of each sequence, then per tile load this CTA's partial S and bulk-copy it
 // into the peer's receive buffer, one 32-token half at a time), warps 4..7 softmax (one thread
 // per row: it adds the peer's partial from the receive buffer to its own from tensor memory),
-// warp 8 TMA producer, warp 9 MMA issuer (one thread).
+// warp 8 TMA producer, warp 9 MMA issuer (one thread); warps 10 and 11 exist to help warp 8
+// gather tiles token by token with cp.async when pages do not hold whole tiles.
 // Tensor memory: O [0, 256), two S buffers [256, 384) with P(j) written over S(j) as bf16 pairs,
 // and q's latent half [384, 512) as the A operand of the score product.  Keeping q there leaves
 // shared memory for four 36 KB KV stages next to the exchange buffers.  Every wait is bounded.
