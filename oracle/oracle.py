@@ -26,7 +26,11 @@ VARIANTS = {"gqa": 0, "gta": 1, "gla": 2}
 
 
 def build(force: bool = False) -> str:
-    """Compile oracle.c with plain gcc -O2 -fopenmp (no fast-math)."""
+    """Compile oracle.c with plain gcc -O2 -fopenmp (no fast-math).  KVD_ORACLE_LIB names an
+    already-built library to use instead (the tests point it at deliberately broken copies to
+    show that the pins catch them)."""
+    if os.environ.get("KVD_ORACLE_LIB"):
+        return os.environ["KVD_ORACLE_LIB"]
     if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
         return _LIB
     os.makedirs(os.path.dirname(_LIB), exist_ok=True)
