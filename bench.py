@@ -7,8 +7,12 @@ synthetic workload.  Default workload: GTA decode, batch 32, q_len 1, h_q 32,
 8 tied KV groups, d_h 128, shared RoPE slice 64, contexts uniform in
 [1024, 8192], page size 64, shuffled block table.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gta|gqa|mla|gla2] [--qlen L]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload W] [--qlen L] [--page-size S]
+  python bench.py --workload gta_prefix|gta_prefix_long [--cascade]   # shared-prefix decode
+  python bench.py --workload append_gta|append_gqa|append_mla|append_gla2 [--tokens N]   # cache append + RoPE
   python bench.py --impl reference ...   # the fp64 CPU oracle timed on this host
+
+Decode workloads W: gta (default), gqa, mla, gla2, gla8, gta_tiny, gta_prefix, gta_prefix_long.
 
 Multi-GPU: the path has no exchange step (sequences are independent), so N GPUs
 run N independent replicas of the step (weak scaling, no collective on the data
@@ -225,7 +229,8 @@ def run_reference(args, inp, cfg, rank):
 
 
 # ----------------------------------------------------------------------------- cache append
-APPEND_SHAPES = {  # per token: (plain heads, plain dim, rope slices, d_r, rope inside the key heads)
+APPEND_SHAPES = {  # per new token, GTA/GLA: `heads` state rows of `dim` and one d_r rope slice;
+    # GQA: `heads` K rows (the last d_r dims of each rotated) and `heads` V rows of `dim`
     "append_gta": dict(kind="gta", heads=8, dim=128, d_r=64),
     "append_gqa": dict(kind="gqa", heads=8, dim=128, d_r=128),
     "append_mla": dict(kind="gla", heads=1, dim=512, d_r=64),
