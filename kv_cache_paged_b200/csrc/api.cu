@@ -13,6 +13,24 @@
 
 using namespace kvd;
 
+namespace kvd {
+// SM count of the calling thread's current device, looked up once per device.
+int num_sms_current() {
+    static std::atomic<int> cache[64];  // zero-initialised (static storage)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    const bool cached = dev >= 0 && dev < 64;
+    if (cached) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    if (cached) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+}  // namespace kvd
+
 namespace {
 
 // Dynamic shared memory the decode kernels may ask for (the SM's 227 KB less
@@ -53,17 +71,6 @@ bool encode(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, 
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), dims, strides, box,
               es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int num_sms_current() {
-    static int cache[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-    if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-    if (dev >= 0 && dev < 64) cache[dev] = n;
-    return n;
 }
 
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }

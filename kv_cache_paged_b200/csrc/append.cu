@@ -16,6 +16,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "kernels.h"
 #include "kvappend.h"
 
 namespace kvd {
@@ -123,13 +124,8 @@ bool aligned16(const void *p) { return p && ((uintptr_t)p & 15u) == 0; }
 int launch_append(AppendArgs &a, int rope_w, double base, cudaStream_t st) {
     if (a.N == 0) return KVD_OK;
     fill_theta(a.theta, rope_w, base);
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return KVD_ERR_CUDA;
-    }
+    const int sms = num_sms_current();
+    if (sms <= 0) return KVD_ERR_CUDA;
     const int blocks = std::min((a.N + 7) / 8, sms * 8);
     append_kernel<<<(unsigned)blocks, 256, 0, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? KVD_OK : KVD_ERR_CUDA;

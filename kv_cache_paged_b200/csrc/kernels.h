@@ -8,6 +8,9 @@
 
 namespace kvd {
 
+// SM count of the calling thread's current device (cached per device; -1 on a CUDA error).
+int num_sms_current();
+
 constexpr int MAX_STAGES = 8;
 
 // Test knobs (kvd_debug_set): make the first tile's copy never start so that the
