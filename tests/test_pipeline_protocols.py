@@ -1,7 +1,7 @@
-"""Barrier protocols of the tcgen05 kernels, modelled on the CPU.
+"""Barrier protocols of the decode kernels, modelled on the CPU.
 
-Every warp role of the GLA kernel (latent_decode.cu) and of the MLA CTA-pair kernel
-(latent_pair.cu) is a coroutine that waits on and arrives at its mbarriers in the order the
+Every warp role of the GQA/GTA kernel (group_decode.cu: box loads or gathered tiles), of the
+GLA kernel (latent_decode.cu) and of the MLA CTA-pair kernel (latent_pair.cu) is a coroutine that waits on and arrives at its mbarriers in the order the
 kernel does; TMA copies, bulk copies to the peer CTA and tcgen05.commit arrivals complete later,
 in random order.  Random schedules over several segment patterns and stage counts must all
 finish (no stall), and no wait may find its barrier two or more phases past the phase it waits
@@ -191,7 +191,50 @@ def mla_pair_model(seed, segs, nstage):
     return schedule(gens, events, rnd)
 
 
+def group_model(seed, segs, nstage, gpc=8, gather_warps=0):
+    """group_decode_kernel: one producer warp (or `gather_warps` warps whose every lane arrives
+    once its copies land) fills an n-stage ring; each of the gpc consumer warps frees a stage
+    after its MMAs on it."""
+    rnd = random.Random(seed)
+    events = []
+    full_count = 32 * gather_warps if gather_warps else 1
+    full = [Bar(f"full{s}", full_count) for s in range(nstage)]
+    empty = [Bar(f"empty{s}", gpc) for s in range(nstage)]
+    ntiles = sum(segs)
+
+    def box_producer():
+        for it in range(ntiles):
+            st = it % nstage
+            yield from wait(lambda: it < nstage or empty[st].ready(it // nstage - 1))
+            full[st].expect_tx(1)
+            events.append(lambda st=st: full[st].complete_tx(1))
+
+    def gather_producer():
+        for it in range(ntiles):
+            st = it % nstage
+            yield from wait(lambda: it < nstage or empty[st].ready(it // nstage - 1))
+            for _ in range(32):  # every lane's cp.async arrive fires when its copies land
+                events.append(lambda st=st: full[st].arrive())
+
+    def consumer():
+        for it in range(ntiles):
+            yield from wait(lambda: full[it % nstage].ready(it // nstage))
+            empty[it % nstage].arrive()
+
+    prods = [gather_producer() for _ in range(gather_warps)] if gather_warps else [box_producer()]
+    return schedule(prods + [consumer() for _ in range(gpc)], events, rnd)
+
+
 SEGS = [(3, 1, 4), (1, 1, 1, 1), (7,), (2, 5), (1, 9, 1)]
+
+
+@pytest.mark.parametrize("gather_warps", [0, 4])
+@pytest.mark.parametrize("nstage", [2, 3])
+def test_group_protocol_finishes_without_parity_aliasing(gather_warps, nstage):
+    ALIAS.clear()
+    for seed in range(25):
+        assert group_model(seed, (5, 2, 6), nstage, gather_warps=gather_warps) == "ok", seed
+    assert not ALIAS, ALIAS[:5]
 
 
 @pytest.mark.parametrize("model", [gla_model, mla_pair_model], ids=["gla", "mla_pair"])
