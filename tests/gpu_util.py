@@ -41,13 +41,14 @@ def to_np(out, lse):
 
 
 def assert_close(out, lse, ref_out, ref_lse, what="", stress=False):
-    """The benchmark spec tolerance: max abs <= 1e-2, mean abs <= 1e-3 on out; |lse| <= 1e-3.
+    """The stated tolerance: max abs <= 1e-2, mean abs <= 1e-3 on out; |lse| <= 1e-3.
 
-    ``stress``: for synthetic stress inputs whose outputs are O(1) (one or two visible
-    tokens with N(0,1) values, near one-hot softmax) the bf16 result itself cannot hold
-    1e-2 absolute: rounding out to bf16 costs up to 2^-9 |out| and the bf16 weights of
-    P another 2^-9 max|v - out|.  There the per-element bound is 1e-2 + 2^-9 |ref|
-    (the output-rounding term made explicit); mean and lse bounds are unchanged.
+    ``stress`` (opt-in, only for cases whose rows see one or two tokens, so that |out| is
+    O(1) and reaches past 2.5): the bf16 result itself cannot always hold 1e-2 absolute
+    there, because rounding the output to bf16 costs up to 2^-9 |out| and the bf16 weights
+    of P up to 2^-9 max|v - out| more.  Such a case gets the per-element bound
+    1e-2 + 2^-9 |ref| (the output-rounding term made explicit); mean and lse bounds are
+    unchanged.  Every other test uses the flat bound.
     """
     assert out.shape == ref_out.shape, (out.shape, ref_out.shape)
     assert np.isfinite(out).all(), f"{what}: non-finite output"

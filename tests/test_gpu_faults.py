@@ -25,6 +25,8 @@ CASES = {
     "gta": dict(variant="gta", B=3, L=1, h_q=32, h_kv=8, d=128, d_r=64, page_size=64, seqlens=[300, 70, 500]),
     "gla2": dict(variant="gla", B=2, L=2, h_q=128, h_kv=2, d=256, d_r=64, page_size=64, seqlens=[200, 90],
                  scale=0.07),
+    "gla2_q1": dict(variant="gla", B=2, L=1, h_q=128, h_kv=2, d=256, d_r=64, page_size=64, seqlens=[300, 90],
+                    scale=0.07),
     "mla": dict(variant="gla", B=2, L=1, h_q=128, h_kv=1, d=512, d_r=64, page_size=64, seqlens=[200, 90],
                 scale=0.07, latent_scale=0.1),
 }
@@ -45,4 +47,4 @@ def test_missing_copy_times_out_and_context_survives(cuda_device, short_waits, n
     assert binding.read_device_error(ws) == 0
     o, l = gu.to_np(out, lse)
     ref_o, ref_l, _ = orc.decode_inputs(inp)
-    gu.assert_close(o, l, ref_o, ref_l, f"{name} after a timed-out call", stress=True)
+    gu.assert_close(o, l, ref_o, ref_l, f"{name} after a timed-out call")

@@ -10,9 +10,8 @@ from tests.indexing import decode_digits, make_delta_problem
 pytestmark = pytest.mark.gpu
 
 
-def check(inp, num_parts=0, b_sample=None, what="", stress=True):
-    """Workload tests pass stress=False (plain the benchmark spec bound); the synthetic edge and
-    stress shapes use the magnitude-aware bound of gpu_util.assert_close."""
+def check(inp, num_parts=0, b_sample=None, what="", stress=False):
+    """Against the oracle with the flat bound (stress: see gpu_util.assert_close)."""
     out, lse = gu.run_gpu(inp, num_parts=num_parts)
     o, l = gu.to_np(out, lse)
     if b_sample is not None:
@@ -38,7 +37,8 @@ def test_mla_small(cuda_device, L):
 
 @pytest.mark.parametrize("L", [1, 2, 4])
 def test_gla2_small(cuda_device, L):
-    check(small(2, 256, L=L, seqlens=[L, 97, 300]), what=f"GLA-2 L={L}")
+    # stress bound: the first sequence holds exactly L tokens, so its rows see one to L tokens
+    check(small(2, 256, L=L, seqlens=[L, 97, 300]), what=f"GLA-2 L={L}", stress=True)
 
 
 @pytest.mark.parametrize("h_c,d_c", [(1, 512), (2, 256)])
@@ -73,7 +73,69 @@ def test_latent_empty_sequences(cuda_device):
     o, l = gu.to_np(out, lse)
     assert np.all(o[[0, 2]] == 0) and np.all(np.isneginf(l[[0, 2]]))
     ref_o, ref_l, _ = orc.decode_inputs(inp)
-    gu.assert_close(o, l, ref_o, ref_l, stress=True)
+    gu.assert_close(o, l, ref_o, ref_l)
+
+
+# ----------------------------------------------------------------------------- at most 64 rows per latent head
+# GLA-2 at q_len 1 and GLA-8 up to q_len 4 run on the narrow kernel (96-token tiles, M = 64).
+@pytest.mark.parametrize("num_parts", [1, 3, 50, 148])
+def test_narrow_forced_splits(cuda_device, num_parts):
+    inp = small(2, 256, B=5, L=1, seqlens=("uniform", 1, 1500), seed=211 + num_parts)
+    check(inp, num_parts=num_parts, what=f"GLA-2 L=1 parts={num_parts}")
+
+
+def test_narrow_tile_boundaries(cuda_device):
+    sl = [1, 2, 47, 48, 95, 96, 97, 191, 192, 193, 300]
+    inp = small(2, 256, B=len(sl), L=1, seqlens=sl, seed=223)
+    for parts in (0, 1, 4, 64):
+        # stress bound: the one- and two-token sequences have rows that see one or two tokens
+        check(inp, num_parts=parts, what=f"GLA-2 L=1 tile boundaries parts={parts}", stress=True)
+
+
+@pytest.mark.parametrize("S", [16, 24, 32, 48, 64, 96, 128, 192])
+def test_narrow_box_shapes(cuda_device, S):
+    """Every box size the box path cuts a 96-token tile into (16, 24, 32, 48 tokens, and one box
+    of the whole tile when the page holds whole tiles)."""
+    inp = small(2, 256, B=4, L=1, page_size=S, seqlens=("uniform", 30, 700), seed=229 + S)
+    check(inp, num_parts=5, what=f"GLA-2 L=1 S={S}")
+
+
+@pytest.mark.parametrize("h_c,h_q,L", [(4, 32, 3), (8, 128, 1), (2, 8, 1), (1, 64, 1)])
+def test_narrow_row_spreads(cuda_device, h_c, h_q, L):
+    """R = 24, 16, 4 and 64 rows per latent head: 6, 4, 1 and 16 rows per lane quadrant."""
+    inp = small(h_c, 256, h_q=h_q, L=L, seqlens=("uniform", L + 8, 500), seed=233 + h_c + L)
+    check(inp, num_parts=3, what=f"h_c={h_c} h_q={h_q} L={L}")
+
+
+def test_narrow_peaky_softmax(cuda_device):
+    inp = small(2, 256, L=1, seqlens=("uniform", 16, 2000), seed=239)
+    inp.scale *= 8
+    check(inp, num_parts=9)
+
+
+def test_narrow_empty_sequences(cuda_device):
+    inp = small(2, 256, B=4, L=1, seqlens=[0, 70, 0, 5], seed=241)
+    out, lse = gu.run_gpu(inp, num_parts=3)
+    o, l = gu.to_np(out, lse)
+    assert np.all(o[[0, 2]] == 0) and np.all(np.isneginf(l[[0, 2]]))
+    ref_o, ref_l, _ = orc.decode_inputs(inp)
+    gu.assert_close(o, l, ref_o, ref_l)
+
+
+def test_narrow_page_permutation_bit_identical(cuda_device):
+    import torch
+    inp = small(2, 256, B=4, L=1, seqlens=("uniform", 1, 800), seed=251)
+    out1, lse1 = gu.run_gpu(inp)
+    perm = np.random.default_rng(3).permutation(inp.num_pages)
+    inv = np.argsort(perm)
+    for k in inp.caches:
+        inp.caches[k] = np.ascontiguousarray(inp.caches[k][inv])
+    bt = inp.block_table.copy()
+    bt[bt >= 0] = perm[bt[bt >= 0]]
+    inp.block_table = bt
+    out2, lse2 = gu.run_gpu(inp)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(lse1, lse2)
 
 
 # ----------------------------------------------------------------------------- indexing
@@ -102,19 +164,39 @@ def test_latent_page_permutation_bit_identical(cuda_device):
 
 
 # ----------------------------------------------------------------------------- full workloads (sampled)
+def check_full(inp, b_sample, what):
+    """A sample of sequences (always including the longest) against the oracle, plus every
+    sequence against a one-part run of the same kernel: a split or slot error on an unsampled
+    sequence changes its result against the unsplit one."""
+    import torch
+    sel = sorted(set(int(b) for b in b_sample) | {int(np.argmax(inp.seqlens))})
+    dev = gu.to_dev(inp)
+    out, lse = gu.run_gpu(inp, dev=dev)
+    o, l = gu.to_np(out, lse)
+    ref_o, ref_l, _ = orc.decode_inputs(inp, b_list=np.asarray(sel, dtype=np.int32))
+    gu.assert_close(o[sel], l[sel], ref_o, ref_l, what)
+    out1, lse1 = gu.run_gpu(inp, dev=dev, num_parts=1)
+    o1, l1 = gu.to_np(out1, lse1)
+    # the split result and the unsplit one: both within the oracle bound of the exact result,
+    # so within twice that of each other; every row and every sequence is compared
+    assert np.isfinite(o).all() and np.array_equal(np.isfinite(l), np.isfinite(l1)), what
+    assert np.abs(o - o1).max() <= 2 * gu.TOL_MAX_ABS, f"{what}: split vs unsplit {np.abs(o - o1).max():.3e}"
+    fin = np.isfinite(l1)
+    assert np.abs(l[fin] - l1[fin]).max() <= 2 * gu.TOL_LSE, what
+
+
 @pytest.mark.parametrize("L", [1, 2])
 def test_mla_workload_full_size(cuda_device, L):
-    """B 64, h_q 128, one 512-dim latent head + 64 rope, contexts U[4096, 32768]; 6 sequences checked."""
-    inp = wl.make_workload("mla", L=L)
-    check(inp, b_sample=[0, 7, 19, 33, 48, 63], what=f"MLA workload L={L}", stress=False)
+    """B 64, h_q 128, one 512-dim latent head + 64 rope, contexts U[4096, 32768]; 6 sequences and
+    the longest checked against the oracle, every sequence against the unsplit run."""
+    check_full(wl.make_workload("mla", L=L), [0, 7, 19, 33, 48, 63], f"MLA workload L={L}")
 
 
 @pytest.mark.parametrize("L", [1, 2, 4])
 def test_gla2_workload_full_size(cuda_device, L):
-    """B 128, h_q 128 over two 256-dim latent heads + 64 rope, lognormal contexts; 6 sequences checked."""
-    inp = wl.make_workload("gla2", L=L)
-    longest = int(np.argmax(inp.seqlens))
-    check(inp, b_sample=[0, 5, 40, 77, 127, longest], what=f"GLA-2 workload L={L}", stress=False)
+    """B 128, h_q 128 over two 256-dim latent heads + 64 rope, lognormal contexts; 6 sequences and
+    the longest checked against the oracle, every sequence against the unsplit run."""
+    check_full(wl.make_workload("gla2", L=L), [0, 5, 40, 77, 127], f"GLA-2 workload L={L}")
 
 
 @pytest.mark.parametrize("L", [1, 2, 3, 4, 8])

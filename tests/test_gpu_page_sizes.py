@@ -24,7 +24,7 @@ def check(inp, num_parts=0, what=""):
     out, lse = gu.run_gpu(inp, num_parts=num_parts)
     o, l = gu.to_np(out, lse)
     ref_o, ref_l, _ = orc.decode_inputs(inp)
-    gu.assert_close(o, l, ref_o, ref_l, what or inp.name, stress=True)
+    gu.assert_close(o, l, ref_o, ref_l, what or inp.name)
 
 
 @pytest.mark.parametrize("variant", ["gta", "gqa"])
@@ -46,7 +46,7 @@ def test_page_size_one_short_and_empty_sequences(cuda_device):
     o, l = gu.to_np(out, lse)
     assert np.all(o[1] == 0) and np.all(np.isneginf(l[1]))
     ref_o, ref_l, _ = orc.decode_inputs(inp)
-    gu.assert_close(o, l, ref_o, ref_l, "S=1 short", stress=True)
+    gu.assert_close(o, l, ref_o, ref_l, "S=1 short")
 
 
 @pytest.mark.parametrize("variant", ["gqa", "gta"])

@@ -30,7 +30,7 @@ def test_shared_prefix_block_tables(cuda_device, variant, num_parts):
     out, lse = gu.run_gpu(inp, num_parts=num_parts)
     o, l = gu.to_np(out, lse)
     ref_o, ref_l, _ = orc.decode_inputs(inp)
-    gu.assert_close(o, l, ref_o, ref_l, f"{variant} shared prefix", stress=True)
+    gu.assert_close(o, l, ref_o, ref_l, f"{variant} shared prefix")
 
 
 def _sub(inp, table, seqlens):
@@ -61,7 +61,7 @@ def test_cascade_prefix_then_continuation(cuda_device, variant):
     o, l = binding.merge_states(o1, l1, o2, l2)
     torch.cuda.synchronize()
     ref_o, ref_l, _ = orc.decode_inputs(inp)
-    gu.assert_close(*gu.to_np(o, l), ref_o, ref_l, f"{variant} cascade", stress=True)
+    gu.assert_close(*gu.to_np(o, l), ref_o, ref_l, f"{variant} cascade")
 
 
 def test_merge_states_matches_oracle_combine(cuda_device):
@@ -130,7 +130,7 @@ def test_batched_prefix_decode(cuda_device, L, num_parts):
     inp = prefix_inputs("gta", B=8, prefix=P, L=L, seed=70 + L)
     out, lse = _prefix_gpu(inp, gu.to_dev(inp), P, num_parts)
     ref_o, ref_l = _prefix_only_ref(inp, P)
-    gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, f"prefix-only L={L}", stress=True)
+    gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, f"prefix-only L={L}")
 
 
 @pytest.mark.parametrize("S,P", [(1, 77), (16, 96), (64, 64)])
@@ -138,7 +138,7 @@ def test_batched_prefix_decode_page_sizes(cuda_device, S, P):
     inp = prefix_inputs("gta", B=6, prefix=P, S=S, seed=80 + S)
     out, lse = _prefix_gpu(inp, gu.to_dev(inp), P)
     ref_o, ref_l = _prefix_only_ref(inp, P)
-    gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, f"prefix-only S={S}", stress=True)
+    gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, f"prefix-only S={S}")
 
 
 def test_cascade_batched_prefix_then_continuation(cuda_device):
@@ -156,7 +156,7 @@ def test_cascade_batched_prefix_then_continuation(cuda_device):
     o, l = binding.merge_states(o1, l1, o2, l2)
     torch.cuda.synchronize()
     ref_o, ref_l, _ = orc.decode_inputs(inp)
-    gu.assert_close(*gu.to_np(o, l), ref_o, ref_l, "batched prefix cascade", stress=True)
+    gu.assert_close(*gu.to_np(o, l), ref_o, ref_l, "batched prefix cascade")
 
 
 def test_gta_prefix_workload_cascade(cuda_device):
@@ -184,7 +184,7 @@ def test_batched_prefix_more_than_128_rows(cuda_device):
     inp = prefix_inputs("gta", B=48, prefix=P, seed=95)
     out, lse = _prefix_gpu(inp, gu.to_dev(inp), P)
     ref_o, ref_l = _prefix_only_ref(inp, P)
-    gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, "prefix-only 192 rows", stress=True)
+    gu.assert_close(*gu.to_np(out, lse), ref_o, ref_l, "prefix-only 192 rows")
 
 
 def test_batched_prefix_empty_prefix(cuda_device):
