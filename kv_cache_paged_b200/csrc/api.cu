@@ -250,6 +250,9 @@ constexpr size_t LATENT_STATIC_SMEM = 4096;
 struct LatentPlan {
     int spread;  // rows per lane quadrant when the rows are spread (0: not spread)
     bool gather;
+    bool narrow;  // at most 64 rows per latent head of width 256: the narrow kernel
+    int tile;     // tokens per plan tile
+    int box_tok;  // narrow kernel, box path: tokens per TMA box
     LatentShape shape;
     bool pair;
     int n_rt, n_vc, n_sub, parts, nstage, rb;
@@ -294,12 +297,34 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
                 break;
             }
     lp->rb = lp->spread ? lp->spread : (g < 128 ? g : 128);
-    const size_t fixed = SMEM_PER_BLOCK - LATENT_STATIC_SMEM - 1024 - sh.q_bytes - sh.p_bytes;
-    int nstage = (int)(fixed / sh.stage_bytes);
-    if (nstage > MAX_STAGES) nstage = MAX_STAGES;
-    if (nstage < 2) return KVD_ERR_UNSUPPORTED_SHAPE;
-    lp->nstage = nstage;
-    lp->smem = 1024 + sh.q_bytes + (size_t)nstage * sh.stage_bytes + sh.p_bytes;
+    lp->tile = sh.tok;
+    lp->box_tok = 0;
+    lp->narrow = !lp->pair && p->d_c == 256 && R <= 64;
+    if (lp->narrow) {
+        // rows spread over the four lane quadrants, ceil(R / 4) each; the tile is cut into boxes
+        // of the largest size that divides both the tile and the page (at least 16 tokens), else
+        // gathered token by token
+        lp->spread = (int)((R + 3) / 4);
+        lp->tile = narrow_tile_tokens();
+        int gcd = lp->tile, b2 = p->page_size;
+        while (b2) {
+            const int t = gcd % b2;
+            gcd = b2;
+            b2 = t;
+        }
+        lp->box_tok = gcd >= 16 ? gcd : 0;
+        lp->gather = lp->box_tok == 0;
+        lp->nstage = 0;
+        lp->smem = narrow_smem_bytes();
+    }
+    if (!lp->narrow) {
+        const size_t fixed = SMEM_PER_BLOCK - LATENT_STATIC_SMEM - 1024 - sh.q_bytes - sh.p_bytes;
+        int nstage = (int)(fixed / sh.stage_bytes);
+        if (nstage > MAX_STAGES) nstage = MAX_STAGES;
+        if (nstage < 2) return KVD_ERR_UNSUPPORTED_SHAPE;
+        lp->nstage = nstage;
+        lp->smem = 1024 + sh.q_bytes + (size_t)nstage * sh.stage_bytes + sh.p_bytes;
+    }
     int parts = p->num_parts;
     if (parts == 0) {
         const int sms = num_sms_current();
@@ -325,29 +350,48 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     const int kch = d_qk / 64;
     const cuuint64_t tokens = (cuuint64_t)p->num_pages * p->page_size;
     CUtensorMap qm, lm, rm;
-    {
-        cuuint64_t dims[3] = {64, (cuuint64_t)p->B * p->L * p->h_q, (cuuint64_t)kch};
-        cuuint64_t strides[2] = {(cuuint64_t)d_qk * 2, 128};
-        cuuint32_t box[3] = {64, (cuuint32_t)lp.rb, 1};
-        if (!encode(&qm, p->q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
-    }
-    if (lp.gather) {
-        memset(&lm, 0, sizeof(lm));  // gathered tiles are copied with cp.async: no cache maps
+    if (lp.narrow) {
+        memset(&qm, 0, sizeof(qm));  // q rows are copied by the kernel's softmax warps
+        memset(&lm, 0, sizeof(lm));
         memset(&rm, 0, sizeof(rm));
-    } else {
-        {
+        if (!lp.gather) {
+            const cuuint32_t nch = lp.box_tok == lp.tile ? (cuuint32_t)(p->d_c / 64) : 1u;
             cuuint64_t dims[3] = {64, tokens, (cuuint64_t)p->h_c * p->d_c / 64};
             cuuint64_t strides[2] = {(cuuint64_t)p->h_c * p->d_c * 2, 128};
-            cuuint32_t box[3] = {64, (cuuint32_t)lp.shape.tok, (cuuint32_t)(p->d_c / 64)};
+            cuuint32_t box[3] = {64, (cuuint32_t)lp.box_tok, nch};
             if (!encode(&lm, p->latent_cache, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
                 return KVD_ERR_CUDA;
-        }
-        {
-            cuuint64_t dims[2] = {64, tokens};
-            cuuint64_t strides[1] = {128};
-            cuuint32_t box[2] = {64, (cuuint32_t)lp.shape.tok};
-            if (!encode(&rm, p->rope_cache, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            cuuint64_t rdims[2] = {64, tokens};
+            cuuint64_t rstrides[1] = {128};
+            cuuint32_t rbox[2] = {64, (cuuint32_t)lp.box_tok};
+            if (!encode(&rm, p->rope_cache, 2, rdims, rstrides, rbox, CU_TENSOR_MAP_SWIZZLE_128B))
                 return KVD_ERR_CUDA;
+        }
+    } else {
+        {
+            cuuint64_t dims[3] = {64, (cuuint64_t)p->B * p->L * p->h_q, (cuuint64_t)kch};
+            cuuint64_t strides[2] = {(cuuint64_t)d_qk * 2, 128};
+            cuuint32_t box[3] = {64, (cuuint32_t)lp.rb, 1};
+            if (!encode(&qm, p->q, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return KVD_ERR_CUDA;
+        }
+        if (lp.gather) {
+            memset(&lm, 0, sizeof(lm));  // gathered tiles are copied with cp.async: no cache maps
+            memset(&rm, 0, sizeof(rm));
+        } else {
+            {
+                cuuint64_t dims[3] = {64, tokens, (cuuint64_t)p->h_c * p->d_c / 64};
+                cuuint64_t strides[2] = {(cuuint64_t)p->h_c * p->d_c * 2, 128};
+                cuuint32_t box[3] = {64, (cuuint32_t)lp.shape.tok, (cuuint32_t)(p->d_c / 64)};
+                if (!encode(&lm, p->latent_cache, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                    return KVD_ERR_CUDA;
+            }
+            {
+                cuuint64_t dims[2] = {64, tokens};
+                cuuint64_t strides[1] = {128};
+                cuuint32_t box[2] = {64, (cuuint32_t)lp.shape.tok};
+                if (!encode(&rm, p->rope_cache, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+                    return KVD_ERR_CUDA;
+            }
         }
     }
     const size_t slots = (size_t)p->B + lp.parts - 1;
@@ -373,6 +417,7 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     a.n_rt = lp.n_rt;
     a.row_spread = lp.spread;
     a.noncausal = 0;
+    a.box_tok = lp.box_tok;
     a.gather = lp.gather ? 1 : 0;
     a.cache0 = p->latent_cache;
     a.cache1 = p->rope_cache;
@@ -409,6 +454,8 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
         }
         if (launch_mla_pair(qm, qrm, lm2, rm2, a, lp.parts * lp.n_sub * 2, lp.smem, st) != cudaSuccess)
             return KVD_ERR_CUDA;
+    } else if (lp.narrow) {
+        if (launch_gla_narrow(lm, rm, a, lp.parts * lp.n_sub, st) != cudaSuccess) return KVD_ERR_CUDA;
     } else if (launch_latent_decode(p->d_c, qm, lm, rm, a, lp.parts * lp.n_sub, lp.smem, st) != cudaSuccess) {
         return KVD_ERR_CUDA;
     }
@@ -422,7 +469,7 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     c.lse = p->lse;
     c.B = p->B;
     c.L = p->L;
-    c.tile = lp.shape.tok;
+    c.tile = lp.tile;
     c.max_tokens = p->max_pages * p->page_size;
     c.parts = lp.parts;
     c.rows = (int)rows;
@@ -594,6 +641,7 @@ int kvd_gta_prefix_decode(const kvd_gta_params *p, void *ws, size_t ws_bytes, kv
     a.n_rt = pp.n_rt;
     a.row_spread = 0;
     a.noncausal = 1;
+    a.box_tok = 0;
     a.gather = pp.gather ? 1 : 0;
     a.cache0 = p->tied_cache;
     a.cache1 = p->rope_cache;

@@ -59,6 +59,7 @@ struct LatentArgs {
     int row_spread;  // <= 64 rows spread over the TMEM lane quadrants: rows per quadrant (0: off)
     int gather;      // pages hold fewer tokens than a tile (or not a multiple): rows copied token by token
     int noncausal;   // every row sees all T tokens (a shared prefix attended by all query rows)
+    int box_tok;     // narrow kernel: tokens per TMA box (divides the tile and the page)
     const void *cache0, *cache1;  // latent and rope caches (the gathered path reads them directly)
     int parts;
     int nstage;
@@ -84,6 +85,13 @@ cudaError_t launch_latent_decode(int d_c, const CUtensorMap &qm, const CUtensorM
 LatentShape tied_prefix_shape();
 cudaError_t launch_tied_prefix(const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
                                const LatentArgs &a, int grid, size_t smem, cudaStream_t st);
+
+// GLA with at most 64 query rows per latent head (latent_narrow.cu): tiles of
+// narrow_tile_tokens() tokens, M = 64 MMAs, q in shared memory; no q tensor map.
+int narrow_tile_tokens();
+size_t narrow_smem_bytes();
+cudaError_t launch_gla_narrow(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid,
+                              cudaStream_t st);
 
 // d_c = 512 (MLA): CTA pairs splitting the key dimension (latent_pair.cu).
 uint32_t mla_pair_fixed_smem();   // q half + the exchange buffer
