@@ -160,9 +160,10 @@ int kvd_gla_decode(const kvd_gla_params *p, void *workspace, size_t workspace_by
  * what kvd_gta_decode() computes, with the workspace in a fixed 8 MiB device
  * array inside the library (held by every GPU that loads the library until the
  * process exits).  It allocates and frees nothing.
- *   - The first call on each device looks up that array's device address with
- *     that device current (and clears its error word); make that first call
- *     before any stream capture.
+ *   - Every call looks up that array's device address in the current context
+ *     (a host-side lookup; the first one on a device also loads the library's
+ *     device code there, so make the first call on each device before any
+ *     stream capture).
  *   - Calls whose split partials need more than 8 MiB (see
  *     kvd_gta_workspace_size) are rejected with KVD_ERR_WORKSPACE_TOO_SMALL and
  *     launch nothing.

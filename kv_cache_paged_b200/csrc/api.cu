@@ -797,35 +797,20 @@ namespace {
 constexpr size_t NOALLOC_WS_BYTES = 8u << 20;  // 8 MiB
 static __device__ __align__(256) uint8_t g_noalloc_ws[NOALLOC_WS_BYTES];
 
-constexpr int NOALLOC_MAX_DEVICES = 64;
-std::mutex g_noalloc_mu;
-void *g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {nullptr};
-
-// Device address of g_noalloc_ws on the current device.  Host code must not use
+// Device address of g_noalloc_ws in the current context.  Host code must not use
 // the symbol itself as a pointer: on the host it names a stand-in, not device
-// memory.  Done once per device, with that device current.
+// memory.  The address is looked up on every call (a host-side table lookup once
+// the module is loaded), so a context that was reset and recreated gets the new
+// array's address rather than a stale one.  The first lookup on a device loads
+// the library's device code there.
 void *noalloc_workspace(int *status) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || !p) {
         *status = KVD_ERR_CUDA;
         return nullptr;
     }
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_ws) != cudaSuccess || !p) {
-            *status = KVD_ERR_CUDA;
-            return nullptr;
-        }
-        // The error word at the head of the workspace only collects flags; start it at zero.
-        if (cudaMemset(p, 0, WS_HEADER) != cudaSuccess) {
-            *status = KVD_ERR_CUDA;
-            return nullptr;
-        }
-        g_noalloc_ptr[dev] = p;
-    }
     *status = KVD_OK;
-    return g_noalloc_ptr[dev];
+    return p;
 }
 
 }  // namespace
