@@ -3,16 +3,17 @@
 
 A step is one call of the library's decode entry point (device-side split
 planning, the decode kernel and the LSE-combine kernel) over one batch of the
-synthetic workload.  Default workload: GTA decode, batch 32, q_len 1, h_q 32,
-8 tied KV groups, d_h 128, shared RoPE slice 64, contexts uniform in
-[1024, 8192], page size 64, shuffled block table.
+synthetic workload.  Default workload: GLA-2 decode (the largest configuration
+that fits one GPU), batch 128, q_len 1, h_q 128 over two 256-wide latent heads
+plus one shared 64-wide RoPE key, lognormal contexts (median 8192, capped at
+65536), page size 64, shuffled block table.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload W] [--qlen L] [--page-size S]
   python bench.py --workload gta_prefix|gta_prefix_long [--cascade]   # shared-prefix decode
   python bench.py --workload append_gta|append_gqa|append_mla|append_gla2 [--tokens N]   # cache append + RoPE
   python bench.py --impl reference ...   # the fp64 CPU oracle timed on this host
 
-Decode workloads W: gta (default), gqa, mla, gla2, gla8, gta_tiny, gta_prefix, gta_prefix_long.
+Decode workloads W: gla2 (default), gta, gqa, mla, gla8, gta_tiny, gta_prefix, gta_prefix_long.
 
 Multi-GPU: the path has no exchange step (sequences are independent), so N GPUs
 run N independent replicas of the step (weak scaling, no collective on the data
@@ -182,14 +183,14 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- oracle timing
-def oracle_sample(inp, budget_s):
-    """Time the fp64 oracle on a prefix of the batch sized to about budget_s seconds of CPU work.
-    Returns (seconds, fraction of the step's work, threads, sequences)."""
+def oracle_sample(inp, budget_s, threads=0):
+    """Time the fp64 oracle on a prefix of the batch sized to about budget_s seconds of CPU work
+    (threads 0: every core).  Returns (seconds, fraction of the step's work, threads, sequences)."""
     from oracle import oracle as orc
     work = np.maximum(inp.seqlens.astype(np.float64), 0)
     total = work.sum()
     t0 = time.perf_counter()
-    _, _, threads = orc.decode_inputs(inp, b_list=np.array([0], np.int32))
+    _, _, threads = orc.decode_inputs(inp, b_list=np.array([0], np.int32), threads=threads)
     t1 = time.perf_counter() - t0
     per_tok = t1 / max(work[0], 1)
     n, acc = 0, 0.0
@@ -199,7 +200,7 @@ def oracle_sample(inp, budget_s):
     n = max(n, 1)
     bl = np.arange(n, dtype=np.int32)
     t0 = time.perf_counter()
-    _, _, threads = orc.decode_inputs(inp, b_list=bl)
+    _, _, threads = orc.decode_inputs(inp, b_list=bl, threads=threads)
     dt = time.perf_counter() - t0
     return dt, float(work[:n].sum() / total), threads, n
 
@@ -384,7 +385,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="kvd", choices=["kvd", "reference"])
-    ap.add_argument("--workload", default="gta", choices=["gta", "gqa", "mla", "gla2", "gta_tiny", "gta_prefix", "gta_prefix_long", "gla8"] + list(APPEND_SHAPES))
+    ap.add_argument("--workload", default="gla2", choices=["gta", "gqa", "mla", "gla2", "gta_tiny", "gta_prefix", "gta_prefix_long", "gla8"] + list(APPEND_SHAPES))
     ap.add_argument("--tokens", type=int, default=65536, help="new tokens per call (append workloads)")
     ap.add_argument("--qlen", type=int, default=1)
     ap.add_argument("--page-size", type=int, default=0, help="override the workload's page size (tokens per page)")
@@ -573,6 +574,23 @@ def main():
     if err:
         raise SystemExit(f"device error flags after timing: {err}")
 
+    # read-only calibration of device memory (kvd_read_stream, outside the timed regions): the
+    # best rate at which a stream that only reads can arrive, reported beside the copy peak
+    rbuf = torch.empty(2 << 30, dtype=torch.uint8, device=dev)
+    sink = torch.zeros(1, dtype=torch.int64, device=dev)
+    rd_ms = []
+    with torch.cuda.stream(stream):
+        for i in range(8):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            binding.read_stream(rbuf, sink, stream=stream)
+            b.record(stream)
+            b.synchronize()
+            if i >= 3:
+                rd_ms.append(a.elapsed_time(b))
+    read_gbs = rbuf.numel() / (min(rd_ms) * 1e-3) / 1e9
+    del rbuf
+
     t_step = statistics.mean(step_ms)
     t_kern = statistics.mean(kern_ms)
     t_e2e = statistics.mean(e2e_ms)
@@ -588,6 +606,10 @@ def main():
         achieved = nbytes / (t_kern * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm}
     roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    roof["peak_read"] = read_gbs
+    roof["peak_read_source"] = "kvd_read_stream: best of 5 streaming reads of 2 GiB in this process (GB/s)"
+    if not tensor_bound:
+        roof["frac_read"] = achieved / read_gbs
     roof["kernel"] = KERNEL_NAMES[variant_kind]
     roof["kernel_us"] = t_kern * 1e3
     # the committed ncu traffic was taken on the workload's own page size
@@ -622,6 +644,12 @@ def main():
                                 "kind": "oracle",
                                 "sample": f"first {n} of {inp.B} sequences ({frac:.3f} of the step's work), "
                                           f"{reps} run(s) in {total:.1f} s, mean scaled to the whole step"}
+        # the same oracle on one thread, on a smaller sample
+        dt1, frac1, _, n1 = oracle_sample(inp, args.cpu_budget / 3, threads=1)
+        line["cpu_baseline"]["single_thread"] = {
+            "value": dt1 / frac1 * 1e6, "unit": UNIT, "cores": 1,
+            "sample": f"first {n1} of {inp.B} sequences ({frac1:.4f} of the step's work) in {dt1:.1f} s, "
+                      f"scaled to the whole step"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:

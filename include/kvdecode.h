@@ -250,6 +250,18 @@ int kvd_debug_set(int knob, long long value);
  */
 int kvd_profile_events(void *before_main, void *after_main);
 
+/*
+ * Measurement helper (no counterpart in the paper): reads `bytes` of device memory at
+ * `buf` once with streaming 16-byte loads on `stream` (grid: blocks_per_sm x the SM count,
+ * 512 threads each) and writes nothing but, practically never, an increment of *sink
+ * (device memory).  Timed with events around it, it gives the read-only rate of the
+ * device memory, the ceiling a decode kernel that only reads the KV cache streams
+ * against.  `buf` 16-byte aligned, `bytes` a multiple of 16; KVD_ERR_INVALID_ARG
+ * otherwise.  Asynchronous; allocates nothing.
+ */
+int kvd_read_stream(const void *buf, size_t bytes, unsigned long long *sink, int blocks_per_sm,
+                    kvd_stream_t stream);
+
 /* Number of SMs of the current device (the default part count), or a negative code. */
 int kvd_num_sms(void);
 

@@ -104,6 +104,8 @@ def lib():
             L.kvd_read_device_error.restype = ctypes.c_int
             L.kvd_read_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
             L.kvd_num_sms.restype = ctypes.c_int
+            L.kvd_read_stream.restype = ctypes.c_int
+            L.kvd_read_stream.argtypes = [_vp, ctypes.c_size_t, _vp, ctypes.c_int, _vp]
             L.kvd_profile_events.restype = ctypes.c_int
             L.kvd_profile_events.argtypes = [_vp, _vp]
             L.kvd_debug_set.restype = ctypes.c_int
@@ -298,6 +300,13 @@ def profile_events(before=None, after=None):
     b = ctypes.c_void_p(before.cuda_event) if before is not None else None
     a = ctypes.c_void_p(after.cuda_event) if after is not None else None
     _check("kvd_profile_events", lib().kvd_profile_events(b, a))
+
+
+def read_stream(buf, sink, blocks_per_sm=4, stream=None):
+    """Stream-read every byte of the CUDA tensor `buf` once (kvd_read_stream); `sink` is a
+    one-element int64 CUDA tensor the kernel may write."""
+    _check("kvd_read_stream", lib().kvd_read_stream(_vp(buf.data_ptr()), buf.numel() * buf.element_size(),
+                                                     _vp(sink.data_ptr()), int(blocks_per_sm), _stream_ptr(stream)))
 
 
 def debug_set(knob, value):
