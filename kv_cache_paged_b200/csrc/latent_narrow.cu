@@ -46,6 +46,7 @@ constexpr int NSMX = 4;     // softmax warps
 constexpr int NGATHER = 3;  // gather warps (0, 2, 3)
 constexpr int NTHREADS = 32 * (4 + NSMX);
 constexpr float RESCALE_LOG2 = 8.f;
+constexpr int PF = 2;       // tiles ahead of the load that the producer prefetches into L2
 
 template <int TOK>
 struct NarrowCfg {
@@ -71,22 +72,24 @@ struct NarrowCfg {
 template <int NS>
 __device__ __forceinline__ void load_half_row(uint32_t taddr, float (&s)[NS]) {
     if constexpr (NS == 48) {
-        float a[32], b[16];
-        tmem_ld16x2_32<48>(taddr, a);
-        tmem_ld16x2_16<48>(taddr + 32, b);
+        uint32_t a[32], b[16];
+        tmem_ld16x2_32_nw<48>(taddr, a);
+        tmem_ld16x2_16_nw<48>(taddr + 32, b);
+        tmem_ld_wait();
 #pragma unroll
-        for (int k = 0; k < 32; ++k) s[k] = a[k];
+        for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(a[k]);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) s[32 + k] = b[k];
+        for (int k = 0; k < 16; ++k) s[32 + k] = __uint_as_float(b[k]);
     } else {
         static_assert(NS == 64, "half rows of 48 or 64 scores");
-        float a[32], b[32];
-        tmem_ld16x2_32<64>(taddr, a);
-        tmem_ld16x2_32<64>(taddr + 32, b);
+        uint32_t a[32], b[32];
+        tmem_ld16x2_32_nw<64>(taddr, a);
+        tmem_ld16x2_32_nw<64>(taddr + 32, b);
+        tmem_ld_wait();
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-            s[k] = a[k];
-            s[32 + k] = b[k];
+            s[k] = __uint_as_float(a[k]);
+            s[32 + k] = __uint_as_float(b[k]);
         }
     }
 }
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncthreads();
         const int nseg = nseg_sh;
 
-        if (warp == 0 || (a.gather && (warp == 2 || warp == 3))) {
+        if (warp == 0 || warp == 2 || warp == 3) {
             // ================================================================ producer(s)
             const int gw = warp == 0 ? 0 : warp - 1;
             const uint64_t pol = policy_evict_first();
@@ -261,33 +264,59 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     continue;
                 }
                 // box path: a tile is nbox boxes of box_tok tokens, each inside one page; boxes
-                // that start at or past T are not loaded (their rows are masked and zeroed)
+                // that start at or past T are not loaded (their rows are masked and zeroed).  The
+                // three warps 0, 2, 3 issue the boxes together (box k by warp k % 3, lane k / 3):
+                // a TMA instruction costs its warp ~0.1k cycles of issue per active lane, and a
+                // tile's 5 nbox copies from one warp fell behind the stream
                 const int box_tok = a.box_tok;
                 const int nbox = TOK / box_tok;
-                auto box_row = [&](int t, int k) -> int {  // cache row of box k of tile t (lane-local)
-                    const int tok = t * TOK + k * box_tok;
-                    if (k >= nbox || tok >= T) return -1;
-                    int pg = __ldg(bt + tok / a.page_size);
-                    if (pg < 0 || pg >= a.num_pages) {
-                        set_error(a.err, DEVERR_BAD_PAGE);
-                        pg = 0;
-                    }
-                    return pg * a.page_size + tok % a.page_size;
+                const int kbox = gw + NGATHER * lane;  // this lane's box of every tile
+                // block-table entries are read two tiles ahead of their use, so that their latency
+                // overlaps the stage waits; NO_BOX marks a box past T_b
+                constexpr int NO_BOX = -2147483647 - 1;
+                auto raw_entry = [&](int t) -> int {
+                    const int tok = t * TOK + kbox * box_tok;
+                    return (t < sg.t1 && kbox < nbox && tok < T) ? __ldg(bt + tok / a.page_size) : NO_BOX;
                 };
-                int nxt = box_row(sg.t0, lane);
+                auto cache_row = [&](int raw, int t) -> int {  // cache row of this lane's box of tile t
+                    if (raw == NO_BOX) return -1;
+                    if (raw < 0 || raw >= a.num_pages) {
+                        set_error(a.err, DEVERR_BAD_PAGE);
+                        raw = 0;
+                    }
+                    return raw * a.page_size + (t * TOK + kbox * box_tok) % a.page_size;
+                };
+                // warp 0 also brings the pages of tile t + PF into L2 when it loads tile t, so that
+                // their load a stage release later finds them there: whole pages (every latent head
+                // and the rope rows) with one untiled bulk prefetch each, by the first latent head's
+                // CTA only (the others read the same pages at about the same time)
+                const bool pf_warp = warp == 0 && c == 0;
+                const size_t lat_page = (size_t)a.page_size * a.h_c * C::DC * 2, rope_page = (size_t)a.page_size * 128;
+                int pf_next_page = -1;  // logical page index prefetched next (pages already done: below)
+                auto raw_page = [&](int t) -> int {  // lane j: the j-th page of tile t
+                    const int p0 = t * TOK / a.page_size, p1 = (min(t * TOK + TOK, T) - 1) / a.page_size;
+                    return (pf_warp && t < sg.t1 && p0 + lane <= p1) ? __ldg(bt + p0 + lane) : NO_BOX;
+                };
+                int raw_ld = raw_entry(sg.t0), raw_nx = raw_entry(sg.t0 + 1);
+                int raw_pf = raw_page(sg.t0 + PF), raw_pf_nx = raw_page(sg.t0 + PF + 1);
                 for (int t = sg.t0; t < sg.t1 && !stop; ++t) {
-                    const int row = nxt;
-                    if (t + 1 < sg.t1) nxt = box_row(t + 1, lane);
+                    const int row = cache_row(raw_ld, t);
+                    const int pf = raw_pf;
+                    raw_ld = raw_nx;
+                    raw_nx = raw_entry(t + 2);
+                    raw_pf = raw_pf_nx;
+                    raw_pf_nx = raw_page(t + PF + 2);
                     const uint32_t stage = p_issued % NST;
                     if (!mbar_wait_warp(&empty_bar[stage], ((p_issued / NST) & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
                         stop = true;
                         break;
                     }
-                    const int nb = min(nbox, (T - t * TOK + box_tok - 1) / box_tok);
-                    if (lane == 0) mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)(nb * box_tok * C::DQK * 2));
-                    __syncwarp();
+                    if (warp == 0 && lane == 0) {
+                        const int nb = min(nbox, (T - t * TOK + box_tok - 1) / box_tok);
+                        mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)(nb * box_tok * C::DQK * 2));
+                    }
                     if (row >= 0 && (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0)) {
-                        uint8_t *st = stage_s + (size_t)stage * C::STAGE + (size_t)lane * box_tok * 128;
+                        uint8_t *st = stage_s + (size_t)stage * C::STAGE + (size_t)kbox * box_tok * 128;
                         if (box_tok == TOK) {  // one box of all four latent chunks
                             tma_load_3d(st, &latmap, &full_bar[stage], 0, row, c * C::NV, pol);
                         } else {
@@ -297,6 +326,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         }
                         // the rope rows are read by every latent head's CTA: no evict-first hint
                         tma_load_2d(st + C::NV * C::CHUNK, &ropemap, &full_bar[stage], 0, row, pol_rope);
+                    }
+                    if (pf_warp && t + PF < sg.t1) {
+                        // the pages of tile t + PF not prefetched yet (a page can span two tiles)
+                        const int p0 = (t + PF) * TOK / a.page_size;
+                        const int p1 = (min((t + PF) * TOK + TOK, T) - 1) / a.page_size;
+                        const int pg = pf < 0 || pf >= a.num_pages ? 0 : pf;
+                        if (p0 + lane <= p1 && p0 + lane >= pf_next_page) {
+                            bulk_prefetch_l2((const uint8_t *)a.cache0 + (size_t)pg * lat_page, (uint32_t)lat_page);
+                            bulk_prefetch_l2((const uint8_t *)a.cache1 + (size_t)pg * rope_page, (uint32_t)rope_page);
+                        }
+                        pf_next_page = p1 + 1;
                     }
                     ++p_issued;
                 }
