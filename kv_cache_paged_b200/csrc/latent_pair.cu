@@ -57,6 +57,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     __shared__ uint64_t qfull_bar, qtm_bar, qempty_bar, pfull_bar[P_NSB], end_bar;
     __shared__ uint64_t sfull_bar[P_NSB], sread_bar[P_NSB];
     __shared__ uint64_t xfull_bar[2], xfree_bar[2];
+    // teardown drain: psent_sh[w][h] = halves h the peer's send warp w copied into this CTA;
+    // xseen_sh[h] = phases of xfull_bar[h] this CTA has seen complete
+    __shared__ uint32_t psent_sh[4][2], xseen_sh[2];
     __shared__ Seg segs[PMAXSEG];
     __shared__ int nseg_sh, more_sh;
     __shared__ volatile int abort_sh;
@@ -106,6 +109,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
             mbar_arrive_expect_tx(&xfull_bar[h], P_XHALF);  // armed for the first tile
         }
         abort_sh = 0;
+        for (int k = 0; k < 8; ++k) psent_sh[k / 2][k % 2] = 0;
+        xseen_sh[0] = xseen_sh[1] = 0;
         fence_mbar_init();
     }
     if (warp == W_MMA) tmem_alloc(&tmem_sh, 512);
@@ -126,6 +131,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     uint32_t m_tile = 0, m_q = 0;
     uint32_t x_tile = 0, x_s = 0, x_pv = 0;            // softmax
     uint32_t e_t = 0, e_q = 0;                          // send
+    uint32_t sent[2] = {0, 0};                          // send: halves copied to the peer
 
     for (int skip = 0;; skip += PMAXSEG) {
         if (warp == W_PROD) {
@@ -394,6 +400,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
                         if (lane == 0)
                             bulk_copy_to_peer(peer_recv + h * P_XHALF + warp * 4096,
                                               smem_u32(send_s + h * P_XHALF) + warp * 4096, 4096, peer_xfull[h]);
+                        ++sent[h];
                     }
                 }
             }
@@ -449,7 +456,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
                             break;
                         }
                         // the phase is complete: arm the next tile's before any warp frees the buffer
-                        if (threadIdx.x == 128) mbar_arrive_expect_tx(&xfull_bar[h], P_XHALF);
+                        if (threadIdx.x == 128) {
+                            mbar_arrive_expect_tx(&xfull_bar[h], P_XHALF);
+                            *(volatile uint32_t *)&xseen_sh[h] = x_s + 1;
+                        }
                         const uint32_t row = smem_u32(recv_s + h * P_XHALF) + r * 128;
 #pragma unroll
                         for (int c8 = 0; c8 < 8; ++c8) {
@@ -603,9 +613,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
         umma_commit(&end_bar);
         mbar_wait_one(&end_bar, 0, &never, nullptr, lim_ns);
     }
+    // Teardown.  A CTA that gave up early (a wait ran out) may still have one of the peer's bulk
+    // copies landing in its receive buffer: the peer copies a tile's half only after this CTA
+    // freed the previous tile's, so at most the half of tile xseen_sh[h] can be in flight, from
+    // the send warps whose count passes it.  Each send warp tells the peer how many halves it
+    // copied; the receiver completes the bytes of the copies that were never issued and waits
+    // (bounded) for the issued ones, and only then may either CTA exit.
+    if (warp < 4 && lane == 0)
+        for (int h = 0; h < 2; ++h)
+            asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(mapa_shared(smem_u32(&psent_sh[warp][h]), peer)),
+                         "r"(sent[h])
+                         : "memory");
     tc_fence_before();
     __syncthreads();
-    cluster_sync();  // the peer no longer writes into this CTA's shared memory
+    cluster_sync();  // the peer's send counts are visible; nobody sends any more
+    if (threadIdx.x == 0) {
+        volatile int never = 0;
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t f = xseen_sh[h];
+            uint32_t n = 0;
+            for (int w = 0; w < 4; ++w) n += psent_sh[w][h] > f ? 1u : 0u;
+            if (n > 0) {
+                if (n < 4) mbar_complete_tx(&xfull_bar[h], (4 - n) * 4096);
+                mbar_wait_one(&xfull_bar[h], f & 1, &never, nullptr, lim_ns);
+            }
+        }
+    }
+    __syncthreads();
+    cluster_sync();  // every copy into either CTA's shared memory has landed
     tc_fence_after();
     if (warp == W_MMA) tmem_dealloc(tmem, 512);
 }

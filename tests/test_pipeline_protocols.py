@@ -269,3 +269,119 @@ def test_model_detects_a_missing_arrival():
         return schedule(gens, events, rnd, limit=20000)
 
     assert short(0, (3,), 2) == "stuck"
+
+
+def mla_exchange_abort_model(seed, ntiles, abort_cta, abort_tiles, drain=True):
+    """The partial-score exchange of mla_pair_kernel when one CTA gives up early.
+
+    Per CTA, four send warps copy each tile's two halves into the peer (a copy lands later, in
+    random order) once the peer has freed the previous tile's half; four softmax warps wait for
+    a half, the first of them arms the next phase and records it (xseen), and all free the half.
+    In CTA `abort_cta` softmax warp w stops before tile abort_tiles[w] (a bounded wait that ran
+    out).  Every wait is bounded: when nothing can move, all waiting warps give up.  Once every
+    warp has stopped, copies still in flight stay in flight; then (with `drain`) the teardown
+    runs as in the kernel: each CTA completes the bytes of the copies the peer never issued for
+    tile xseen[h] and waits for the issued ones, landing copies only while it waits.  Returns the
+    copies still in flight when the CTAs would exit and whether a drain wait would have run out."""
+    rnd = random.Random(seed)
+    events = []
+    C = []
+    for k in range(2):
+        c = {"xfull": [Bar(f"xfull{k}{h}", 1) for h in range(2)],
+             "xfree": [Bar(f"xfree{k}{h}", 4) for h in range(2)],
+             "sent": [[0, 0] for _ in range(4)], "xseen": [0, 0], "inflight": [0, 0]}
+        for h in range(2):
+            c["xfull"][h].expect_tx(4)
+        C.append(c)
+    stop = [False]
+
+    def land(k, h):
+        C[k]["inflight"][h] -= 1
+        C[k]["xfull"][h].complete_tx(1)
+
+    def send(k, w):
+        c, p = C[k], C[k ^ 1]
+        for e in range(ntiles):
+            for h in range(2):
+                while not (e == 0 or c["xfree"][h].ready(e - 1)):
+                    if stop[0]:
+                        return
+                    yield
+                p["inflight"][h] += 1
+                events.append(lambda h=h: land(k ^ 1, h))
+                c["sent"][w][h] += 1
+
+    def softmax(k, w):
+        c, p = C[k], C[k ^ 1]
+        for x in range(min(abort_tiles[w] if k == abort_cta else ntiles, ntiles)):
+            for h in range(2):
+                while not c["xfull"][h].ready(x):
+                    if stop[0]:
+                        return
+                    yield
+                if w == 0:
+                    c["xfull"][h].expect_tx(4)
+                    c["xseen"][h] = x + 1
+                p["xfree"][h].arrive()
+
+    alive = []
+    for k in range(2):
+        alive += [send(k, w) for w in range(4)] + [softmax(k, w) for w in range(4)]
+    idle = 0
+    while alive:
+        if events and rnd.random() < 0.4:
+            events.pop(rnd.randrange(len(events)))()
+            idle = 0
+            continue
+        i = rnd.randrange(len(alive))
+        try:
+            next(alive[i])
+            idle += 1
+        except StopIteration:
+            alive.pop(i)
+            idle = 0
+        if idle > 40 * (len(alive) + 1) and not events:
+            stop[0] = True  # nothing can move: every bounded wait runs out
+    timed_out = False
+    if drain:
+        for k in range(2):
+            c, p = C[k], C[k ^ 1]
+            for h in range(2):
+                f = c["xseen"][h]
+                n = sum(1 for w in range(4) if p["sent"][w][h] > f)
+                if n:
+                    if n < 4:
+                        c["xfull"][h].complete_tx(4 - n)
+                    while not c["xfull"][h].ready(f):
+                        if not events:
+                            timed_out = True
+                            break
+                        events.pop(rnd.randrange(len(events)))()
+    return [c["inflight"][h] for c in C for h in range(2)], timed_out
+
+
+def _abort_cases():
+    for seed in range(300):
+        rnd = random.Random(1000 + seed)
+        ntiles = rnd.randint(1, 6)
+        base = rnd.randint(0, ntiles)
+        yield seed, ntiles, [max(0, min(ntiles, base + rnd.randint(-1, 1))) for _ in range(4)]
+
+
+@pytest.mark.parametrize("abort_cta", [0, 1])
+def test_pair_teardown_drains_the_peers_copies(abort_cta):
+    """One CTA of the pair gives up mid-stream (its softmax warps at different tiles); after the
+    teardown drain no bulk copy into either CTA's shared memory is still in flight, and no drain
+    wait runs out."""
+    for seed, ntiles, tiles in _abort_cases():
+        inflight, timed_out = mla_exchange_abort_model(seed, ntiles, abort_cta, tiles)
+        assert inflight == [0, 0, 0, 0], (seed, ntiles, tiles, inflight)
+        assert not timed_out, (seed, ntiles, tiles)
+
+
+def test_pair_teardown_without_the_drain_can_exit_under_a_copy():
+    """The check is not vacuous: without the drain some of the same schedules reach the exit with
+    a copy into a CTA's shared memory still in flight."""
+    hits = sum(any(mla_exchange_abort_model(seed, ntiles, 0, tiles, drain=False)[0])
+               for seed, ntiles, tiles in _abort_cases())
+    assert hits > 0
