@@ -45,9 +45,20 @@ FALLBACK_HBM_GBS, FALLBACK_TFLOPS = 6650.0, 1590.0
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 KERNEL_SOURCES = {"group": ["kv_cache_paged_b200/csrc/group_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"],
                   "latent": ["kv_cache_paged_b200/csrc/latent_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"],
+                  "narrow": ["kv_cache_paged_b200/csrc/latent_narrow.cu", "kv_cache_paged_b200/csrc/common.cuh"],
                   "pair": ["kv_cache_paged_b200/csrc/latent_pair.cu", "kv_cache_paged_b200/csrc/common.cuh"],
                   "append": ["kv_cache_paged_b200/csrc/append.cu", "kv_cache_paged_b200/csrc/common.cuh"]}
-KERNEL_NAMES = {"group": "group_decode_kernel", "latent": "latent_decode_kernel", "pair": "mla_pair_kernel"}
+KERNEL_NAMES = {"group": "group_decode_kernel", "latent": "latent_decode_kernel", "narrow": "gla_narrow_kernel",
+                "pair": "mla_pair_kernel"}
+
+
+def kernel_kind(inp):
+    """Which decode kernel the library runs for these inputs (mirrors the dispatch in csrc/api.cu)."""
+    if inp.variant != "gla":
+        return "group"
+    if inp.d == 512:
+        return "pair"
+    return "narrow" if (inp.h_q // inp.h_kv) * inp.L <= 64 and inp.d == 256 else "latent"
 
 
 def describe(inp):
@@ -597,7 +608,7 @@ def main():
     t_step, t_kern, t_e2e = max_over_ranks([t_step, t_kern, t_e2e], pg, device=dev)
 
     hbm, tfl, peak_src = load_peaks()
-    variant_kind = ("pair" if inp.d == 512 else "latent") if inp.variant == "gla" else "group"
+    variant_kind = kernel_kind(inp)
     tensor_bound = flops / (tfl * 1e12) > nbytes / (hbm * 1e9)
     if tensor_bound:
         achieved = flops / (t_kern * 1e-3) / 1e12
