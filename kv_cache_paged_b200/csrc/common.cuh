@@ -82,25 +82,42 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bits) {
 
 // Warp-cooperative plan walk.  Every lane of the calling warp must call it with
 // the same arguments.  Calls emit(seg) on lane 0 for each segment of part c, in
-// order, up to the end of the part; returns N (total tiles).
+// order, up to the end of the part; returns N (total tiles).  The sequence lengths
+// are read PLAN_K per lane at a time, all loads in flight together, and the first
+// 32 PLAN_K tile counts are kept for the second pass: with up to 128 sequences the
+// walk costs one global-memory round trip instead of one per 32 sequences and pass.
+constexpr int PLAN_K = 4;
 template <typename Emit>
 __device__ __forceinline__ int64_t plan_walk(const int32_t *__restrict__ seqlens, int32_t B, int32_t tile,
                                              int32_t max_tokens, int32_t L, int64_t c, int64_t parts,
                                              uint32_t *err, Emit emit) {
     const int lane = threadIdx.x & 31;
     int64_t N = 0;
-    for (int32_t base = 0; base < B; base += 32) {
-        int32_t b = base + lane;
-        int32_t n = 0;
-        if (b < B) {
-            bool bad;
-            int32_t T = clamp_len(__ldg(seqlens + b), max_tokens, L, &bad);
-            if (bad && c == 0) set_error(err, DEVERR_BAD_SEQLEN);
-            n = tiles_of(T, tile);
+    int32_t keep[PLAN_K];  // tile counts of sequences 32 k + lane (the first batch)
+    for (int32_t base = 0; base < B; base += 32 * PLAN_K) {
+        int32_t raw[PLAN_K];
+#pragma unroll
+        for (int k = 0; k < PLAN_K; ++k) {
+            const int32_t b = base + 32 * k + lane;
+            raw[k] = b < B ? __ldg(seqlens + b) : 0;
+        }
+        int32_t tot = 0;
+#pragma unroll
+        for (int k = 0; k < PLAN_K; ++k) {
+            const int32_t b = base + 32 * k + lane;
+            int32_t n = 0;
+            if (b < B) {
+                bool bad;
+                const int32_t T = clamp_len(raw[k], max_tokens, L, &bad);
+                if (bad && c == 0) set_error(err, DEVERR_BAD_SEQLEN);
+                n = tiles_of(T, tile);
+            }
+            if (base == 0) keep[k] = n;
+            tot += n;
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-        N += n;
+        for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        N += tot;
     }
     if (N == 0) return 0;
     if (parts > N) parts = N;
@@ -111,7 +128,13 @@ __device__ __forceinline__ int64_t plan_walk(const int32_t *__restrict__ seqlens
     for (int32_t base = 0; base < B && run < hi; base += 32) {
         int32_t b = base + lane;
         int32_t n = 0;
-        if (b < B) n = tiles_of(clamp_len(__ldg(seqlens + b), max_tokens, L, nullptr), tile);
+        if (base < 32 * PLAN_K) {
+#pragma unroll
+            for (int k = 0; k < PLAN_K; ++k)
+                if (base == 32 * k) n = keep[k];
+        } else if (b < B) {
+            n = tiles_of(clamp_len(__ldg(seqlens + b), max_tokens, L, nullptr), tile);
+        }
         int32_t incl = n;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {

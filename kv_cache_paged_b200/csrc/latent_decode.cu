@@ -270,6 +270,9 @@ __global__ void __launch_bounds__(LTHREADS, 1)
                     // cannot overwrite that P before it is read
                     const uint32_t sb = m_s & 1;
                     tc_fence_after();
+                    // gathered rows were written by cp.async (the generic proxy); the tensor core reads
+                    // them through the async proxy, so order the two before the MMAs
+                    if (a.gather) fence_proxy_async();
                     const uint32_t d = tmem + C::S_COL + sb * TOK;
                     // descriptors advance by (byte offset >> 4) in their low word: one add per MMA
                     const uint64_t dk0 = umma_desc(st0 + stage * C::STAGE, 16, 1024, 2);

@@ -271,6 +271,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
                     const uint32_t stage = gt % nstage;
                     if (!mbar_wait_one(&full_bar[stage], (gt / nstage) & 1, &abort_sh, a.err, lim_ns)) return false;
                     tc_fence_after();
+                    // gathered rows were written by cp.async (the generic proxy); the tensor core reads
+                    // them through the async proxy, so order the two before the MMAs
+                    if (a.gather) fence_proxy_async();
                     const uint32_t d = tmem + P_SCOL + (gt % P_NSB) * PTOK;
                     const uint64_t dk0 = umma_desc(st0 + stage * P_STAGE, 16, 1024, 2);
                     const uint64_t dkr = umma_desc(st0 + stage * P_STAGE + 4 * P_CHUNK, 16, 512, 4);
