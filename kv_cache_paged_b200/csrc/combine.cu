@@ -16,13 +16,10 @@ namespace kvd {
 
 namespace {
 
-constexpr int CROWS = 8;   // rows per CTA
+constexpr int CROWS = 32;  // rows per CTA
 
 __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     __shared__ int first_sh, nsplit_sh;
-
-    // Wait for the decode grid to finish and its partials to be visible.
-    pdl_wait();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x;
@@ -30,14 +27,25 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     const int nrow = min(CROWS, a.rows - row0);
 
     if (warp == 0) {
+        // the sequence's part range from seqlens: PLAN_K lengths per lane per round trip
         int64_t N = 0, cu = 0;
         int32_t nb = 0;
-        for (int base = 0; base < a.B; base += 32) {
-            const int idx = base + lane;
-            int32_t n = 0;
-            if (idx < a.B) n = tiles_of(clamp_len(__ldg(a.seqlens + idx), a.max_tokens, a.L, nullptr), a.tile);
-            int32_t before = idx < b ? n : 0;
-            int32_t mine = idx == b ? n : 0;
+        for (int base = 0; base < a.B; base += 32 * PLAN_K) {
+            int32_t raw[PLAN_K];
+#pragma unroll
+            for (int k = 0; k < PLAN_K; ++k) {
+                const int idx = base + 32 * k + lane;
+                raw[k] = idx < a.B ? __ldg(a.seqlens + idx) : 0;
+            }
+            int32_t n = 0, before = 0, mine = 0;
+#pragma unroll
+            for (int k = 0; k < PLAN_K; ++k) {
+                const int idx = base + 32 * k + lane;
+                const int32_t t = idx < a.B ? tiles_of(clamp_len(raw[k], a.max_tokens, a.L, nullptr), a.tile) : 0;
+                n += t;
+                before += idx < b ? t : 0;
+                mine += idx == b ? t : 0;
+            }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 n += __shfl_xor_sync(0xffffffffu, n, o);
@@ -63,6 +71,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     __syncthreads();
     const int nsplit = nsplit_sh;
     if (nsplit == 1) return;  // the decode kernel wrote this sequence's output itself
+    // The part range above needs only seqlens (an input), so it overlaps the decode grid's tail;
+    // the partials are read only once the decode grid has finished and they are visible.
+    pdl_wait();
     const int first = first_sh;
     const size_t rows = (size_t)a.rows;
 
