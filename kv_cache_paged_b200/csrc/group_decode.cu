@@ -29,10 +29,10 @@ namespace kvd {
 namespace {
 
 constexpr int MAXSEG = 128;
-constexpr int GATHER_WARPS = 4;  // producer warps when tiles are gathered token by token
-
-template <bool TIED, int D, int DR, int NT, int TT>
-__global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
+// GW: producer warps when tiles are gathered token by token (the block has up to 8 + GW warps;
+// box-load launches use one producer warp but keep the GW = 4 bound, so their code is unchanged)
+template <bool TIED, int D, int DR, int NT, int TT, int GW>
+__global__ void __launch_bounds__((8 + GW) * 32, 1)
     group_decode_kernel(const __grid_constant__ CUtensorMap map0, const __grid_constant__ CUtensorMap map1,
                         const GroupArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -54,7 +54,7 @@ __global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nstage; ++s) {
-            mbar_init(&full_bar[s], a.gather ? 32 * GATHER_WARPS : 1);  // gathered: every producer lane
+            mbar_init(&full_bar[s], a.gather ? 32 * GW : 1);  // gathered: every producer lane
             mbar_init(&empty_bar[s], gpc);
         }
         abort_sh = 0;
@@ -94,15 +94,16 @@ __global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
                 const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
                 if (a.gather) {
                     // Pages smaller than a tile (down to one token) or not a multiple of it.  The
-                    // GATHER_WARPS producer warps all walk every tile; warp w copies the tokens
-                    // k = w, w + GATHER_WARPS, ...: one lane per token resolves its cache row
+                    // GW producer warps all walk every tile; warp w copies the tokens
+                    // k = w, w + GW, ...: one lane per token resolves its cache row
                     // (distributed offset calculation, fetched a tile ahead), then the warp copies
                     // each token's row with 16-byte cp.async into the same swizzled layout the box
                     // loads produce (a token's row is contiguous: 32 lanes move 512 consecutive
                     // bytes per instruction).  Every lane arrives on the stage's barrier when its
                     // copies have landed.
                     const int pw = warp - gpc;
-                    constexpr int TPW = TT / GATHER_WARPS;      // tokens per warp and tile
+                    constexpr int TPW = (TT + GW - 1) / GW;     // most tokens a warp takes per tile
+                    const int nkw = (TT - pw + GW - 1) / GW;    // the tokens this warp takes
                     const int T = clamp_len(__ldg(a.seqlens + sg.b), max_tokens, a.L, nullptr);
                     const int nch = gpc * (D / 64);
                     const size_t row_elems = (size_t)a.h_kv * D;
@@ -110,15 +111,15 @@ __global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
                     const __nv_bfloat16 *c1 = (const __nv_bfloat16 *)a.cache1 + (TIED ? 0 : (size_t)z0 * 64);
                     constexpr int RU = TIED ? DR * 2 / 16 : 0;  // 16-byte units of a rope row
                     // token of this lane in tile t (tokens past T_b repeat the last one; masked later)
-                    auto tok_of = [&](int t) { return min(t * TT + pw + GATHER_WARPS * lane, T - 1); };
+                    auto tok_of = [&](int t) { return min(t * TT + pw + GW * lane, T - 1); };
                     int nxt_tok = tok_of(sg.t0);
-                    int nxt_page = lane < TPW ? __ldg(bt + nxt_tok / a.page_size) : 0;
+                    int nxt_page = lane < nkw ? __ldg(bt + nxt_tok / a.page_size) : 0;
                     for (int t = sg.t0; t < sg.t1 && !stop; ++t, ++issued) {
                         const int tok = nxt_tok;
                         int page = nxt_page;
                         if (t + 1 < sg.t1) {
                             nxt_tok = tok_of(t + 1);
-                            if (lane < TPW) nxt_page = __ldg(bt + nxt_tok / a.page_size);
+                            if (lane < nkw) nxt_page = __ldg(bt + nxt_tok / a.page_size);
                         }
                         const uint32_t stage = issued % nstage;
                         if (!mbar_wait_warp(&empty_bar[stage], ((issued / nstage) & 1) ^ 1, &abort_sh, a.err,
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
                             stop = true;
                             break;
                         }
-                        if (lane < TPW && (page < 0 || page >= a.num_pages)) {
+                        if (lane < nkw && (page < 0 || page >= a.num_pages)) {
                             set_error(a.err, DEVERR_BAD_PAGE);
                             page = 0;
                         }
@@ -140,7 +141,8 @@ __global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
                             const int nj = (nch * 8 - lane + 31) / 32;  // this lane's units of a row
 #pragma unroll
                             for (int i = 0; i < TPW; ++i) {
-                                const uint32_t k = (uint32_t)(pw + GATHER_WARPS * i);
+                                if (i >= nkw) break;
+                                const uint32_t k = (uint32_t)(pw + GW * i);
                                 const size_t row = (size_t)__shfl_sync(0xffffffffu, myrow, i);
                                 const uint32_t dst = dst_l + k * 128u + ((c_l ^ (k & 7u)) << 4);
                                 const __nv_bfloat16 *s0 = c0 + row * row_elems + lane * 8;
@@ -153,14 +155,14 @@ __global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
                             }
                             if constexpr (TIED) {
                                 // rope rows, 32 / RU tokens per instruction: lane l copies unit l % RU
-                                // of token pw + GATHER_WARPS (i0 + l / RU)
+                                // of token pw + GW (i0 + l / RU)
                                 const uint32_t ru = (uint32_t)(lane % RU);
 #pragma unroll
                                 for (int i0 = 0; i0 < TPW; i0 += 32 / RU) {
                                     const int i = i0 + lane / RU;
                                     const size_t row = (size_t)__shfl_sync(0xffffffffu, myrow, i & 31);
-                                    if (i < TPW) {
-                                        const uint32_t k = (uint32_t)(pw + GATHER_WARPS * i);
+                                    if (i < nkw) {
+                                        const uint32_t k = (uint32_t)(pw + GW * i);
                                         cp_async16(st + kv_tile + (DR == 64 ? sw128(k, ru) : sw64(k, ru)),
                                                    c1 + row * DR + ru * 8, pol);
                                     }
@@ -492,20 +494,23 @@ __global__ void __launch_bounds__((8 + GATHER_WARPS) * 32, 1)
     }
 }
 
-template <bool TIED, int D, int DR, int NT, int TT>
+template <bool TIED, int D, int DR, int NT, int TT, int GW = 4>
 cudaError_t launch_t(const CUtensorMap &m0, const CUtensorMap &m1, const GroupArgs &a, int grid, size_t smem,
                      cudaStream_t st) {
-    auto k = group_decode_kernel<TIED, D, DR, NT, TT>;
+    auto k = group_decode_kernel<TIED, D, DR, NT, TT, GW>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, (a.gpc + (a.gather ? GATHER_WARPS : 1)) * 32, smem, st>>>(m0, m1, a);
+    k<<<grid, (a.gpc + (a.gather ? GW : 1)) * 32, smem, st>>>(m0, m1, a);
     return cudaGetLastError();
 }
 
 template <bool TIED, int D, int DR>
 cudaError_t launch_nt(int nt, const CUtensorMap &m0, const CUtensorMap &m1, const GroupArgs &a, int grid,
                       size_t smem, cudaStream_t st) {
-    if (a.tile == 32 && nt == 1) return launch_t<TIED, D, DR, 1, 32>(m0, m1, a, grid, smem, st);
+    // gathered 32-token tiles (GTA at small page sizes): six producer warps keep more copies in flight
+    if (a.tile == 32 && nt == 1)
+        return a.gather ? launch_t<TIED, D, DR, 1, 32, 6>(m0, m1, a, grid, smem, st)
+                        : launch_t<TIED, D, DR, 1, 32>(m0, m1, a, grid, smem, st);
     if (a.tile != 16) return cudaErrorInvalidValue;
     switch (nt) {
         case 1: return launch_t<TIED, D, DR, 1, 16>(m0, m1, a, grid, smem, st);

@@ -72,7 +72,7 @@ def group_expected(tied, nch, dr, tt, row_of):
 @pytest.mark.parametrize("tied,d,dr", [(False, 64, 0), (False, 128, 0), (True, 64, 32), (True, 128, 32),
                                        (True, 128, 64), (True, 64, 64)])
 @pytest.mark.parametrize("gpc", [1, 2, 4, 8])
-@pytest.mark.parametrize("tt,gw", [(16, 4), (32, 4)])
+@pytest.mark.parametrize("tt,gw", [(16, 4), (32, 4), (32, 6)])
 def test_group_gather_covers_the_box_layout(tied, d, dr, gpc, tt, gw):
     nch = gpc * d // 64
     row_of = lambda k: 1000 + 7 * k  # distinct rows per token
@@ -107,10 +107,11 @@ def gather_tile(nch, rw, chunk_bytes, k0, kstep, nk, row_of):
     return writes
 
 
-@pytest.mark.parametrize("nch,rw", [(4, 8), (2, 8), (4, 4)])  # GLA d_c 256, GTA prefix d_h 128, MLA half
-@pytest.mark.parametrize("nwarps", [3, 5])
-def test_latent_gather_covers_the_box_layout(nch, rw, nwarps):
-    tok = 64
+@pytest.mark.parametrize("nch,rw,tok", [(4, 8, 64), (2, 8, 64), (4, 4, 64), (4, 8, 96)])  # GLA d_c 256 (64- and
+@pytest.mark.parametrize("nwarps", [3, 5])                                                  # 96-token tiles), GTA
+def test_latent_gather_covers_the_box_layout(nch, rw, tok, nwarps):                          # prefix, MLA half
+    if (tok + nwarps - 1) // nwarps > 32:
+        pytest.skip("one token per gather lane")
     chunk_bytes = tok * 128
     row_of = lambda k: 500 + 3 * k
     writes = {}
