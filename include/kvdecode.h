@@ -215,14 +215,17 @@ int kvd_merge_states(const void *out_a, const float *lse_a, const void *out_b, c
  * exactly as the decode kernels do and writes, for part c, up to `cap` records
  * of 6 int32 {b, tile_begin, tile_end, split_index, num_splits, slot} at
  * segments[c * cap * 6 ...] and the record count at counts[c] (device
- * pointers).  A count above `cap` means records were dropped.
+ * pointers).  A count above `cap` means records were dropped.  seg_cost >= 0:
+ * each non-empty sequence counts as seg_cost extra tiles placed before its
+ * own when the stream is cut into parts of equal size (the GLA kernel for at
+ * most 64 rows per latent head plans with 3, the others with 0).
  */
-int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_tokens, int32_t num_parts,
-             int32_t *segments, int32_t *counts, int32_t cap, kvd_stream_t stream);
+int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t seg_cost, int32_t max_tokens,
+             int32_t num_parts, int32_t *segments, int32_t *counts, int32_t cap, kvd_stream_t stream);
 
 /* The same plan computed on the host from host memory; returns KVD_OK. */
-int kvd_plan_host(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_tokens, int32_t num_parts,
-                  int32_t *segments, int32_t *counts, int32_t cap);
+int kvd_plan_host(const int32_t *seqlens, int32_t B, int32_t tile, int32_t seg_cost, int32_t max_tokens,
+                  int32_t num_parts, int32_t *segments, int32_t *counts, int32_t cap);
 
 /*
  * Synchronises `stream`, reads the workspace's device error word into *flags

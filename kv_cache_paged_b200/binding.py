@@ -98,9 +98,9 @@ def lib():
                 w.restype = ctypes.c_size_t
                 w.argtypes = [ctypes.POINTER(P)]
             L.kvd_plan.restype = ctypes.c_int
-            L.kvd_plan.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp]
+            L.kvd_plan.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp]
             L.kvd_plan_host.restype = ctypes.c_int
-            L.kvd_plan_host.argtypes = [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32]
+            L.kvd_plan_host.argtypes = [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32]
             L.kvd_read_device_error.restype = ctypes.c_int
             L.kvd_read_device_error.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
             L.kvd_num_sms.restype = ctypes.c_int
@@ -271,25 +271,25 @@ def read_device_error(ws, stream=None):
     return flags.value
 
 
-def plan_device(seqlens, tile, max_tokens, num_parts, cap=64, stream=None):
+def plan_device(seqlens, tile, max_tokens, num_parts, cap=64, stream=None, seg_cost=0):
     """Run the device planner; returns (segments int32 [parts, cap, 6], counts [parts]) on the device."""
     torch = _torch()
     segs = torch.full((num_parts, cap, 6), -1, dtype=torch.int32, device=seqlens.device)
     counts = torch.zeros(num_parts, dtype=torch.int32, device=seqlens.device)
-    st = lib().kvd_plan(_dev(seqlens, "seqlens", torch.int32, 1), seqlens.shape[0], tile, max_tokens, num_parts,
+    st = lib().kvd_plan(_dev(seqlens, "seqlens", torch.int32, 1), seqlens.shape[0], tile, seg_cost, max_tokens, num_parts,
                         ctypes.c_void_p(segs.data_ptr()), ctypes.c_void_p(counts.data_ptr()), cap,
                         _stream_ptr(stream))
     _check("kvd_plan", st)
     return segs, counts
 
 
-def plan_host(seqlens, tile, max_tokens, num_parts, cap=64):
+def plan_host(seqlens, tile, max_tokens, num_parts, cap=64, seg_cost=0):
     """The same plan computed on the host (numpy int32 in, numpy arrays out)."""
     import numpy as np
     sl = np.ascontiguousarray(seqlens, dtype=np.int32)
     segs = np.full((num_parts, cap, 6), -1, dtype=np.int32)
     counts = np.zeros(num_parts, dtype=np.int32)
-    st = lib().kvd_plan_host(sl.ctypes.data_as(_vp), sl.shape[0], tile, max_tokens, num_parts,
+    st = lib().kvd_plan_host(sl.ctypes.data_as(_vp), sl.shape[0], tile, seg_cost, max_tokens, num_parts,
                              segs.ctypes.data_as(_vp), counts.ctypes.data_as(_vp), cap)
     _check("kvd_plan_host", st)
     return segs, counts

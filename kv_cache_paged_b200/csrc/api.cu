@@ -206,6 +206,7 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
     a.num_pages = P;
     a.max_pages = max_pages;
     a.tile = gp.tile;
+    a.seg_cost = 0;
     a.gather = gp.gather ? 1 : 0;
     a.cache0 = c0;
     a.cache1 = c1;
@@ -233,6 +234,7 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
     c.B = B;
     c.L = L;
     c.tile = gp.tile;
+    c.seg_cost = 0;
     c.max_tokens = max_pages * S;
     c.parts = gp.parts;
     c.rows = (int)rows;
@@ -253,6 +255,7 @@ struct LatentPlan {
     bool narrow;  // at most 64 rows per latent head of width 256: the narrow kernel
     int tile;     // tokens per plan tile
     int box_tok;  // narrow kernel, box path: tokens per TMA box
+    int seg_cost; // plan: units a segment start costs, in tiles
     LatentShape shape;
     bool pair;
     int n_rt, n_vc, n_sub, parts, nstage, rb;
@@ -299,6 +302,7 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
     lp->rb = lp->spread ? lp->spread : (g < 128 ? g : 128);
     lp->tile = sh.tok;
     lp->box_tok = 0;
+    lp->seg_cost = 0;
     lp->narrow = !lp->pair && p->d_c == 256 && R <= 64;
     if (lp->narrow) {
         // rows spread over the four lane quadrants, ceil(R / 4) each; the tile is cut into boxes
@@ -314,6 +318,7 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
         }
         lp->box_tok = gcd >= 16 ? gcd : 0;
         lp->gather = lp->box_tok == 0;
+        lp->seg_cost = narrow_seg_cost();
         lp->nstage = 0;
         lp->smem = narrow_smem_bytes();
     }
@@ -418,6 +423,7 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     a.row_spread = lp.spread;
     a.noncausal = 0;
     a.box_tok = lp.box_tok;
+    a.seg_cost = lp.seg_cost;
     a.gather = lp.gather ? 1 : 0;
     a.cache0 = p->latent_cache;
     a.cache1 = p->rope_cache;
@@ -470,6 +476,7 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     c.B = p->B;
     c.L = p->L;
     c.tile = lp.tile;
+    c.seg_cost = lp.seg_cost;
     c.max_tokens = p->max_pages * p->page_size;
     c.parts = lp.parts;
     c.rows = (int)rows;
@@ -642,6 +649,7 @@ int kvd_gta_prefix_decode(const kvd_gta_params *p, void *ws, size_t ws_bytes, kv
     a.row_spread = 0;
     a.noncausal = 1;
     a.box_tok = 0;
+    a.seg_cost = 0;
     a.gather = pp.gather ? 1 : 0;
     a.cache0 = p->tied_cache;
     a.cache1 = p->rope_cache;
@@ -662,6 +670,7 @@ int kvd_gta_prefix_decode(const kvd_gta_params *p, void *ws, size_t ws_bytes, kv
     c.B = 1;
     c.L = 1;  // the plan of a non-causal pseudo-sequence (every position sees all tokens)
     c.tile = pp.shape.tok;
+    c.seg_cost = 0;
     c.max_tokens = p->max_pages * p->page_size;
     c.parts = pp.parts;
     c.rows = (int)rows;
@@ -682,30 +691,32 @@ int kvd_merge_states(const void *out_a, const float *lse_a, const void *out_b, c
                : KVD_ERR_CUDA;
 }
 
-int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_tokens, int32_t num_parts,
-             int32_t *segments, int32_t *counts, int32_t cap, kvd_stream_t stream) {
-    if (B < 0 || tile < 1 || max_tokens < 0 || num_parts < 1 || cap < 0) return KVD_ERR_INVALID_ARG;
+int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t seg_cost, int32_t max_tokens,
+             int32_t num_parts, int32_t *segments, int32_t *counts, int32_t cap, kvd_stream_t stream) {
+    if (B < 0 || tile < 1 || seg_cost < 0 || max_tokens < 0 || num_parts < 1 || cap < 0) return KVD_ERR_INVALID_ARG;
     if ((B > 0 && !seqlens) || !counts || (cap > 0 && !segments)) return KVD_ERR_INVALID_ARG;
-    return launch_plan(seqlens, B, tile, max_tokens, 1, num_parts, segments, counts, cap, (cudaStream_t)stream) ==
+    return launch_plan(seqlens, B, tile, seg_cost, max_tokens, 1, num_parts, segments, counts, cap,
+                       (cudaStream_t)stream) ==
                    cudaSuccess
                ? KVD_OK
                : KVD_ERR_CUDA;
 }
 
-int kvd_plan_host(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_tokens, int32_t num_parts,
-                  int32_t *segments, int32_t *counts, int32_t cap) {
-    if (B < 0 || tile < 1 || max_tokens < 0 || num_parts < 1 || cap < 0) return KVD_ERR_INVALID_ARG;
+int kvd_plan_host(const int32_t *seqlens, int32_t B, int32_t tile, int32_t seg_cost, int32_t max_tokens,
+                  int32_t num_parts, int32_t *segments, int32_t *counts, int32_t cap) {
+    if (B < 0 || tile < 1 || seg_cost < 0 || max_tokens < 0 || num_parts < 1 || cap < 0) return KVD_ERR_INVALID_ARG;
     if ((B > 0 && !seqlens) || !counts || (cap > 0 && !segments)) return KVD_ERR_INVALID_ARG;
     int64_t N = 0;
-    for (int b = 0; b < B; ++b) N += tiles_of(clamp_len(seqlens[b], max_tokens, 1, nullptr), tile);
+    for (int b = 0; b < B; ++b) N += units_of(tiles_of(clamp_len(seqlens[b], max_tokens, 1, nullptr), tile), seg_cost);
     const int64_t P = N < num_parts ? N : num_parts;
     for (int c = 0; c < num_parts; ++c) {
         int cnt = 0;
         if (N > 0 && c < P) {
             const int64_t lo = part_begin(c, N, P), hi = part_begin(c + 1, N, P);
-            int64_t cu = 0;
-            for (int b = 0; b < B && cu < hi; ++b) {
+            int64_t run = 0;  // units before sequence b
+            for (int b = 0; b < B && run < hi; ++b) {
                 const int32_t n = tiles_of(clamp_len(seqlens[b], max_tokens, 1, nullptr), tile);
+                const int64_t cu = run + units_of(n, seg_cost) - n;  // the unit of b's first tile
                 if (n > 0 && cu < hi && cu + n > lo) {
                     if (cnt < cap) {
                         Seg s = make_seg(b, cu, n, lo, hi, c, N, P);
@@ -719,7 +730,7 @@ int kvd_plan_host(const int32_t *seqlens, int32_t B, int32_t tile, int32_t max_t
                     }
                     ++cnt;
                 }
-                cu += n;
+                run += units_of(n, seg_cost);
             }
         }
         counts[c] = cnt;

@@ -16,7 +16,7 @@ namespace kvd {
 
 namespace {
 
-constexpr int CROWS = 32;  // rows per CTA
+constexpr int CROWS = 8;   // rows per CTA
 
 __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     __shared__ int first_sh, nsplit_sh;
@@ -42,8 +42,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
             for (int k = 0; k < PLAN_K; ++k) {
                 const int idx = base + 32 * k + lane;
                 const int32_t t = idx < a.B ? tiles_of(clamp_len(raw[k], a.max_tokens, a.L, nullptr), a.tile) : 0;
-                n += t;
-                before += idx < b ? t : 0;
+                const int32_t u = (int32_t)units_of(t, a.seg_cost);
+                n += u;
+                before += idx < b ? u : (idx == b ? u - t : 0);  // up to this sequence's first tile
                 mine += idx == b ? t : 0;
             }
 #pragma unroll
@@ -117,11 +118,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     }
 }
 
-__global__ void plan_kernel(const int32_t *seqlens, int B, int tile, int max_tokens, int L, int parts,
+__global__ void plan_kernel(const int32_t *seqlens, int B, int tile, int seg_cost, int max_tokens, int L, int parts,
                             int32_t *segs, int32_t *counts, int cap) {
     const int c = blockIdx.x;
     int cnt = 0;
-    plan_walk(seqlens, B, tile, max_tokens, L, c, parts, nullptr, [&](const Seg &s) {
+    plan_walk(seqlens, B, tile, seg_cost, max_tokens, L, c, parts, nullptr, [&](const Seg &s) {
         if (cnt < cap) {
             int32_t *o = segs + ((size_t)c * cap + cnt) * 6;
             o[0] = s.b;
@@ -201,9 +202,9 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_plan(const int32_t *seqlens, int B, int tile, int max_tokens, int L, int parts, int32_t *segs,
-                        int32_t *counts, int cap, cudaStream_t st) {
-    plan_kernel<<<parts, 32, 0, st>>>(seqlens, B, tile, max_tokens, L, parts, segs, counts, cap);
+cudaError_t launch_plan(const int32_t *seqlens, int B, int tile, int seg_cost, int max_tokens, int L, int parts,
+                        int32_t *segs, int32_t *counts, int cap, cudaStream_t st) {
+    plan_kernel<<<parts, 32, 0, st>>>(seqlens, B, tile, seg_cost, max_tokens, L, parts, segs, counts, cap);
     return cudaGetLastError();
 }
 

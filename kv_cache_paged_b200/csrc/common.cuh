@@ -80,17 +80,24 @@ __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bits) {
     if (err) atomicOr(err, bits);
 }
 
+// The (sequence, tile) stream, with a cost: every non-empty sequence contributes seg_cost
+// units before its tiles (the fixed work of starting a segment: its q, the pipeline's refill,
+// its epilogue, counted in tiles), so the parts, cut into equal numbers of units, give fewer
+// tiles to a part that starts more sequences.  Sequence b's tiles are the units
+// [cu_b, cu_b + n_b) and its first tile is unit cu_b; seg_cost 0 is the plain tile stream.
+__host__ __device__ inline int64_t units_of(int32_t n, int32_t seg_cost) { return n > 0 ? (int64_t)n + seg_cost : 0; }
+
 // Warp-cooperative plan walk.  Every lane of the calling warp must call it with
 // the same arguments.  Calls emit(seg) on lane 0 for each segment of part c, in
-// order, up to the end of the part; returns N (total tiles).  The sequence lengths
+// order, up to the end of the part; returns N (total units).  The sequence lengths
 // are read PLAN_K per lane at a time, all loads in flight together, and the first
 // 32 PLAN_K tile counts are kept for the second pass: with up to 128 sequences the
 // walk costs one global-memory round trip instead of one per 32 sequences and pass.
 constexpr int PLAN_K = 4;
 template <typename Emit>
 __device__ __forceinline__ int64_t plan_walk(const int32_t *__restrict__ seqlens, int32_t B, int32_t tile,
-                                             int32_t max_tokens, int32_t L, int64_t c, int64_t parts,
-                                             uint32_t *err, Emit emit) {
+                                             int32_t seg_cost, int32_t max_tokens, int32_t L, int64_t c,
+                                             int64_t parts, uint32_t *err, Emit emit) {
     const int lane = threadIdx.x & 31;
     int64_t N = 0;
     int32_t keep[PLAN_K];  // tile counts of sequences 32 k + lane (the first batch)
@@ -113,7 +120,7 @@ __device__ __forceinline__ int64_t plan_walk(const int32_t *__restrict__ seqlens
                 n = tiles_of(T, tile);
             }
             if (base == 0) keep[k] = n;
-            tot += n;
+            tot += (int32_t)units_of(n, seg_cost);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
@@ -135,13 +142,13 @@ __device__ __forceinline__ int64_t plan_walk(const int32_t *__restrict__ seqlens
         } else if (b < B) {
             n = tiles_of(clamp_len(__ldg(seqlens + b), max_tokens, L, nullptr), tile);
         }
-        int32_t incl = n;
+        int32_t incl = (int32_t)units_of(n, seg_cost);
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
-        int64_t cu = run + (incl - n);
+        int64_t cu = run + (incl - n);  // the unit of this sequence's first tile
         bool hit = (b < B) && n > 0 && cu < hi && cu + n > lo;
         uint32_t mask = __ballot_sync(0xffffffffu, hit);
         while (mask) {

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__((8 + GW) * 32, 1)
     for (int skip = 0;; skip += MAXSEG) {
         if (warp == gpc) {
             int cnt = 0;
-            plan_walk(a.seqlens, a.B, TT, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
+            plan_walk(a.seqlens, a.B, TT, a.seg_cost, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
                 if (cnt >= skip && cnt < skip + MAXSEG) segs[cnt - skip] = s;
                 ++cnt;
             });

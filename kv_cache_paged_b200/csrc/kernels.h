@@ -28,6 +28,7 @@ struct GroupArgs {
     uint32_t *err;
     int B, L, h_q, h_kv, page_size, num_pages, max_pages;
     int tile;   // tokens per pipeline stage (16 or 32)
+    int seg_cost;  // plan: units a segment start costs, in tiles
     int gather; // pages hold fewer tokens than a tile (or not a multiple): rows copied token by token
     const void *cache0, *cache1;  // K / tied and V / rope caches (the gathered path reads them directly)
     int gpc;    // KV groups per CTA (consumer warps)
@@ -60,6 +61,7 @@ struct LatentArgs {
     int gather;      // pages hold fewer tokens than a tile (or not a multiple): rows copied token by token
     int noncausal;   // every row sees all T tokens (a shared prefix attended by all query rows)
     int box_tok;     // narrow kernel: tokens per TMA box (divides the tile and the page)
+    int seg_cost;    // plan: units a segment start costs, in tiles
     const void *cache0, *cache1;  // latent and rope caches (the gathered path reads them directly)
     int parts;
     int nstage;
@@ -89,6 +91,7 @@ cudaError_t launch_tied_prefix(const CUtensorMap &qm, const CUtensorMap &lm, con
 // GLA with at most 64 query rows per latent head (latent_narrow.cu): tiles of
 // narrow_tile_tokens() tokens, M = 64 MMAs, q in shared memory; no q tensor map.
 int narrow_tile_tokens();
+int narrow_seg_cost();  // the plan's cost of a segment start, in tiles
 size_t narrow_smem_bytes();
 cudaError_t launch_gla_narrow(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid,
                               cudaStream_t st);
@@ -105,7 +108,7 @@ struct CombineArgs {
     const float *ws_o;
     __nv_bfloat16 *out;
     float *lse;
-    int B, L, tile, max_tokens, parts;
+    int B, L, tile, seg_cost, max_tokens, parts;
     int rows;  // L * h_q
     int d_v;
 };
@@ -118,7 +121,7 @@ cudaError_t launch_merge(const void *out_a, const float *lse_a, const void *out_
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 
 // Writes the plan of every part (see kvd_plan).
-cudaError_t launch_plan(const int32_t *seqlens, int B, int tile, int max_tokens, int L, int parts, int32_t *segs,
-                        int32_t *counts, int cap, cudaStream_t st);
+cudaError_t launch_plan(const int32_t *seqlens, int B, int tile, int seg_cost, int max_tokens, int L, int parts,
+                        int32_t *segs, int32_t *counts, int cap, cudaStream_t st);
 
 }  // namespace kvd

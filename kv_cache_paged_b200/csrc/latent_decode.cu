@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(LTHREADS, 1)
     for (int skip = 0;; skip += LMAXSEG) {
         if (warp == 0) {
             int cnt = 0;
-            plan_walk(a.seqlens, a.B, TOK, max_tokens, a.noncausal ? 1 : a.L, part, a.parts, a.err, [&](const Seg &s) {
+            plan_walk(a.seqlens, a.B, TOK, a.seg_cost, max_tokens, a.noncausal ? 1 : a.L, part, a.parts, a.err, [&](const Seg &s) {
                 if (cnt >= skip && cnt < skip + LMAXSEG) segs[cnt - skip] = s;
                 ++cnt;
             });

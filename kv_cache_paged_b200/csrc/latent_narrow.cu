@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int skip = 0;; skip += NMAXSEG) {
         if (warp == 0) {
             int cnt = 0;
-            plan_walk(a.seqlens, a.B, TOK, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
+            plan_walk(a.seqlens, a.B, TOK, a.seg_cost, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
                 if (cnt >= skip && cnt < skip + NMAXSEG) segs[cnt - skip] = s;
                 ++cnt;
             });
@@ -602,6 +602,10 @@ cudaError_t launch_t(const CUtensorMap &lm, const CUtensorMap &rm, const LatentA
 }  // namespace
 
 int narrow_tile_tokens() { return NARROW_TOK; }
+// A segment start costs the CTA about 4 us (its q copy, the refill of the ring, the epilogue of
+// the segment before it) against ~1.5 us per 96-token tile at the HBM rate: a part that starts
+// six sequences ended ~20 us after the median one when parts were cut by tiles alone.
+int narrow_seg_cost() { return 3; }
 size_t narrow_smem_bytes() { return NarrowCfg<NARROW_TOK>::SMEM; }
 
 cudaError_t launch_gla_narrow(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid,

@@ -136,7 +136,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     for (int skip = 0;; skip += PMAXSEG) {
         if (warp == W_PROD) {
             int cnt = 0;
-            plan_walk(a.seqlens, a.B, PTOK, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
+            plan_walk(a.seqlens, a.B, PTOK, a.seg_cost, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
                 if (cnt >= skip && cnt < skip + PMAXSEG) segs[cnt - skip] = s;
                 ++cnt;
             });

@@ -136,6 +136,53 @@ def test_plan_with_empty_and_tiny_sequences():
         _check_plan(sl, 16, parts)
 
 
+def _plan_reference(seqlens, tile, parts, seg_cost, max_tokens=1 << 30):
+    """The plan written out in Python: non-empty sequence b is seg_cost units followed by its tiles;
+    the unit stream is cut into min(parts, N) equal parts; a part's segment of b is b's tiles inside
+    the part's unit range."""
+    tiles = [-(-min(max(int(t), 0), max_tokens) // tile) for t in seqlens]
+    units = [n + seg_cost if n else 0 for n in tiles]
+    N = sum(units)
+    P = min(parts, N)
+    out = [[] for _ in range(parts)]
+    if N == 0:
+        return out
+    first_unit, run = [], 0
+    for n, u in zip(tiles, units):
+        first_unit.append(run + u - n)
+        run += u
+    part_of = lambda x: ((x + 1) * P - 1) // N
+    for c in range(P):
+        lo, hi = c * N // P, (c + 1) * N // P
+        for b, n in enumerate(tiles):
+            cu = first_unit[b]
+            if n and cu < hi and cu + n > lo:
+                f, l = part_of(cu), part_of(cu + n - 1)
+                out[c].append((b, max(lo, cu) - cu, min(hi, cu + n) - cu, c - f, l - f + 1, b + c))
+    return out
+
+
+@pytest.mark.parametrize("seg_cost", [0, 1, 3, 20])
+@pytest.mark.parametrize("parts", [1, 3, 74, 148, 1000])
+def test_plan_with_a_segment_cost_matches_its_definition(parts, seg_cost):
+    rng = np.random.default_rng(parts + seg_cost)
+    sl = np.clip(np.round(np.exp(rng.normal(np.log(8192), 1.0, 128))), 1, 65536).astype(np.int32)
+    sl[rng.integers(0, 128, 6)] = 0  # a few empty sequences
+    segs, counts = binding.plan_host(sl, 96, 1 << 30, parts, cap=160, seg_cost=seg_cost)
+    ref = _plan_reference(sl, 96, parts, seg_cost)
+    for c in range(parts):
+        got = [tuple(int(x) for x in segs[c, k]) for k in range(int(counts[c]))]
+        assert got == ref[c], (c, got[:3], ref[c][:3])
+    # every tile once, and a part that starts more sequences holds fewer tiles
+    tiles = {}
+    for c in range(parts):
+        for (b, t0, t1, *_r) in ref[c]:
+            tiles.setdefault(b, []).append((t0, t1))
+    for b, n in enumerate(-(-int(t) // 96) for t in sl):
+        got = sorted(tiles.get(b, []))
+        assert sum(t1 - t0 for t0, t1 in got) == n and all(a[1] == z[0] for a, z in zip(got, got[1:]))
+
+
 def test_plan_all_empty():
     segs, counts = binding.plan_host(np.zeros(5, np.int32), 16, 1 << 20, 4)
     assert counts.sum() == 0

@@ -159,9 +159,9 @@ def test_device_plan_equals_host_plan(cuda_device):
     rng = np.random.default_rng(1)
     sl = rng.integers(0, 3000, size=77).astype(np.int32)
     sl[::7] = 0
-    for parts in (1, 13, 148, 500):
-        hs, hc = binding.plan_host(sl, 16, 1 << 20, parts, cap=96)
-        ds, dc = binding.plan_device(torch.from_numpy(sl).cuda(), 16, 1 << 20, parts, cap=96)
+    for parts, seg_cost in ((1, 0), (13, 0), (148, 0), (500, 0), (13, 3), (148, 3), (74, 11)):
+        hs, hc = binding.plan_host(sl, 16, 1 << 20, parts, cap=96, seg_cost=seg_cost)
+        ds, dc = binding.plan_device(torch.from_numpy(sl).cuda(), 16, 1 << 20, parts, cap=96, seg_cost=seg_cost)
         dc = dc.cpu().numpy()
         ds = ds.cpu().numpy()
         assert np.array_equal(hc, dc)
