@@ -218,7 +218,8 @@ int kvd_merge_states(const void *out_a, const float *lse_a, const void *out_b, c
  * pointers).  A count above `cap` means records were dropped.  seg_cost >= 0:
  * each non-empty sequence counts as seg_cost extra tiles placed before its
  * own when the stream is cut into parts of equal size (the GLA kernel for at
- * most 64 rows per latent head plans with 3, the others with 0).
+ * most 64 rows per latent head plans with 3, GTA with 128 / tile, the others
+ * with 0).
  */
 int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t seg_cost, int32_t max_tokens,
              int32_t num_parts, int32_t *segments, int32_t *counts, int32_t cap, kvd_stream_t stream);

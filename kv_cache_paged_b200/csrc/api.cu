@@ -79,6 +79,7 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // ----------------------------------------------------------------------------- GQA / GTA
 struct GroupPlan {
     int gpc, n_sub, parts, nt, nstage, tile;
+    int seg_cost;  // plan: units a segment start costs, in tiles
     bool gather;
     uint32_t stage_bytes, stage_bytes_tx;
     size_t ws_bytes;
@@ -147,6 +148,11 @@ int plan_group(bool tied, const void *q, const void *c0, const void *c1, const i
     gp->nt = nt;
     gp->nstage = nstage;
     gp->tile = tile;
+    // GTA: a segment start (q rows, the ring's refill, the epilogue) costs about as much as
+    // streaming 128 tokens; the split plan counts it (measured on B 32 with 1k..8k contexts:
+    // 68.8 us against 72.7 us without).  GQA streams twice the bytes per token and measured no
+    // gain from it.
+    gp->seg_cost = tied ? 128 / tile : 0;
     gp->gather = gather;
     gp->stage_bytes = stage;
     gp->stage_bytes_tx = tx;
@@ -206,7 +212,7 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
     a.num_pages = P;
     a.max_pages = max_pages;
     a.tile = gp.tile;
-    a.seg_cost = 0;
+    a.seg_cost = gp.seg_cost;
     a.gather = gp.gather ? 1 : 0;
     a.cache0 = c0;
     a.cache1 = c1;
@@ -234,7 +240,7 @@ int run_group(bool tied, const void *q, const void *c0, const void *c1, const in
     c.B = B;
     c.L = L;
     c.tile = gp.tile;
-    c.seg_cost = 0;
+    c.seg_cost = gp.seg_cost;
     c.max_tokens = max_pages * S;
     c.parts = gp.parts;
     c.rows = (int)rows;

@@ -16,9 +16,13 @@ namespace kvd {
 
 namespace {
 
-constexpr int CROWS = 8;   // rows per CTA
+// 4 rows per CTA (one 16-byte column group of one row per thread at d_v 256), loads of 4 parts
+// per round trip, at most 40 registers: 6 CTAs per SM, so that the grid runs in fewer waves
+// once the decode grid has drained (the combine's time is a chain of round trips per CTA)
+constexpr int CROWS = 4;
+constexpr int CPARTS = 4;
 
-__global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
+__global__ void __launch_bounds__(256, 6) combine_kernel(const CombineArgs a) {
     __shared__ int first_sh, nsplit_sh;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -78,25 +82,26 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineArgs a) {
     const int first = first_sh;
     const size_t rows = (size_t)a.rows;
 
-    // One memory round: each thread owns four consecutive outputs of one row and loads that
-    // row's lse and its four columns from every part together, then reduces locally.
+    // Each thread owns four consecutive outputs of one row and loads that row's lse and its four
+    // columns from CPARTS parts per round trip (one round trip for up to CPARTS parts), reducing
+    // locally.
     const int dv4 = a.d_v / 4;
     for (int idx = threadIdx.x; idx < nrow * dv4; idx += blockDim.x) {
         const int r = row0 + idx / dv4, c4 = idx % dv4;
         float mx = -INFINITY, sum = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s0 = 0; s0 < nsplit; s0 += 8) {
-            float ls[8];
-            float4 x[8];
+        for (int s0 = 0; s0 < nsplit; s0 += CPARTS) {
+            float ls[CPARTS];
+            float4 x[CPARTS];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < CPARTS; ++k) {
                 const size_t slot = (size_t)(b + first) + min(s0 + k, nsplit - 1);
                 ls[k] = s0 + k < nsplit ? __ldcs(a.ws_lse + slot * rows + r) : -INFINITY;
                 x[k] = __ldcs((const float4 *)(a.ws_o + (slot * rows + r) * a.d_v) + c4);
             }
             // streaming log-sum-exp over the parts, rescaling what is summed so far
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < CPARTS; ++k) {
                 if (ls[k] == -INFINITY) continue;
                 const float mn = fmaxf(mx, ls[k]);
                 const float sc = mx == -INFINITY ? 0.f : expf(mx - mn);

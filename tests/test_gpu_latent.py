@@ -113,13 +113,91 @@ def test_narrow_peaky_softmax(cuda_device):
     check(inp, num_parts=9)
 
 
-def test_narrow_empty_sequences(cuda_device):
-    inp = small(2, 256, B=4, L=1, seqlens=[0, 70, 0, 5], seed=241)
-    out, lse = gu.run_gpu(inp, num_parts=3)
+def _gla_call(d, inp, out, lse, num_parts, ws, stream=None):
+    from kv_cache_paged_b200 import binding
+    return binding.gla_decode(d["q"], d["latent_cache"], d["rope_cache"], d["block_table"], d["seqlens"], inp.scale,
+                              num_parts=num_parts, out=out, lse=lse, workspace=ws, stream=stream)
+
+
+def _nan_outputs(inp):
+    import torch
+    out = torch.full((inp.B, inp.L, inp.h_q, inp.d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((inp.B, inp.L, inp.h_q), float("nan"), dtype=torch.float32, device="cuda")
+    return out, lse
+
+
+@pytest.mark.parametrize("num_parts", [1, 3, 0])
+def test_narrow_empty_sequences(cuda_device, num_parts):
+    """Empty sequences have no tiles and no part visits them: the combine writes their rows
+    (outputs start as NaN so that nothing passes by chance)."""
+    import torch
+    inp = small(2, 256, B=6, L=1, seqlens=[0, 70, 0, 5, 300, 0], seed=241)
+    d = gu.to_dev(inp)
+    out, lse = _nan_outputs(inp)
+    _gla_call(d, inp, out, lse, num_parts, torch.zeros(1 << 24, dtype=torch.uint8, device="cuda"))
     o, l = gu.to_np(out, lse)
-    assert np.all(o[[0, 2]] == 0) and np.all(np.isneginf(l[[0, 2]]))
+    assert np.all(o[[0, 2, 5]] == 0) and np.all(np.isneginf(l[[0, 2, 5]]))
     ref_o, ref_l, _ = orc.decode_inputs(inp)
     gu.assert_close(o, l, ref_o, ref_l)
+
+
+def test_narrow_all_sequences_empty(cuda_device):
+    import torch
+    inp = small(2, 256, B=3, L=1, seqlens=[0, 0, 0], seed=243)
+    d = gu.to_dev(inp)
+    out, lse = _nan_outputs(inp)
+    _gla_call(d, inp, out, lse, 0, torch.zeros(1 << 24, dtype=torch.uint8, device="cuda"))
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_narrow_split_merge_ignores_stale_workspace(cuda_device):
+    """Arbitrary bytes in the workspace (left by other calls, or never cleared) do not change the
+    result of a split call: every partial the combine reads was written by this call.  Only the
+    error word has to start at zero."""
+    import torch
+    inp = small(2, 256, B=7, L=1, seqlens=("uniform", 200, 3000), seed=245)
+    d = gu.to_dev(inp)
+    clean = torch.zeros(1 << 24, dtype=torch.uint8, device="cuda")
+    ref_out, ref_lse = _nan_outputs(inp)
+    _gla_call(d, inp, ref_out, ref_lse, 23, clean)
+    dirty = torch.randint(0, 256, (1 << 24,), dtype=torch.uint8, device="cuda")
+    dirty[:256] = 0
+    for call in range(3):
+        out, lse = _nan_outputs(inp)
+        _gla_call(d, inp, out, lse, 23, dirty)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16)), f"call {call}"
+        assert torch.equal(lse.view(torch.int32), ref_lse.view(torch.int32)), f"call {call}"
+    o, l = gu.to_np(ref_out, ref_lse)
+    ref_o, ref_l, _ = orc.decode_inputs(inp)
+    gu.assert_close(o, l, ref_o, ref_l)
+
+
+def test_narrow_graph_replay(cuda_device):
+    """A captured split call (decode kernel, then the combine as its programmatic dependent)
+    replays bit for bit."""
+    import torch
+    inp = small(2, 256, B=6, L=1, seqlens=("uniform", 100, 2500), seed=247)
+    d = gu.to_dev(inp)
+    ws = torch.zeros(1 << 24, dtype=torch.uint8, device="cuda")
+    out, lse = _nan_outputs(inp)
+    _gla_call(d, inp, out, lse, 17, ws)   # eager run (also sets kernel attributes)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = out.clone(), lse.clone()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            _gla_call(d, inp, out, lse, 17, ws, stream=s)
+    for replay in range(3):
+        out.fill_(float("nan"))
+        lse.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16)), f"replay {replay}"
+        assert torch.equal(lse.view(torch.int32), ref_lse.view(torch.int32)), f"replay {replay}"
+    from kv_cache_paged_b200 import binding
+    assert binding.read_device_error(ws) == 0
 
 
 def test_narrow_page_permutation_bit_identical(cuda_device):
