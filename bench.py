@@ -491,8 +491,9 @@ def main():
     c0, c1 = caches[names[0]], caches[names[1]]
     launches_per_step = 2  # decode kernel (planning fused in) + LSE combine
 
-    def step(qq, btt, sll):
-        fn(qq, c0, c1, btt, sll, inp.scale, out=out, lse=lse, workspace=ws, stream=stream)
+    def step(qq, btt, sll, oo=None, ll=None):
+        fn(qq, c0, c1, btt, sll, inp.scale, out=out if oo is None else oo, lse=lse if ll is None else ll,
+           workspace=ws, stream=stream)
 
     if args.cascade:
         # cascade decoding of a batch-shared prefix: the prefix once for all rows of a KV group
@@ -513,11 +514,12 @@ def main():
         ws_p = torch.zeros(1 << 28, dtype=torch.uint8, device=dev)
         launches_per_step = 5  # prefix kernel + combine, continuation kernel + combine, merge
 
-        def step(qq, btt, sll):
+        def step(qq, btt, sll, oo=None, ll=None):
             binding.gta_prefix_decode(qq, c0, c1, pre_bt, pre_len, inp.scale, out=out_p, lse=lse_p, workspace=ws_p,
                                       stream=stream)
             binding.gta_decode(qq, c0, c1, btt, sll, inp.scale, out=out_s, lse=lse_s, workspace=ws, stream=stream)
-            binding.merge_states(out_p, lse_p, out_s, lse_s, out=out, lse=lse, stream=stream)
+            binding.merge_states(out_p, lse_p, out_s, lse_s, out=out if oo is None else oo,
+                                 lse=lse if ll is None else ll, stream=stream)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -581,6 +583,47 @@ def main():
             ee[k][1].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = [ee[k][0].elapsed_time(ee[k][1]) for k in range(KE)]
+
+    # the same KE steps as a serving loop runs them: two sets of input and result buffers, the
+    # H2D of step k + 1 and the D2H of step k - 1 on their own streams overlapping step k's
+    # kernels; every step still moves its inputs in and its result out.  Per-step time = the
+    # whole loop (first H2D issued to last D2H done) / KE.
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    in_d2 = [in_d, torch.empty_like(in_d)]
+    views2 = [(q, bt, sl), tuple(in_d2[1][t.data_ptr() - in_d.data_ptr():][:t.numel() * t.element_size()]
+                                 .view(t.dtype).view(t.shape) for t in (q, bt, sl))]
+    res_d2 = [res_d, torch.empty_like(res_d)]
+    outs2 = [(out, lse), (res_d2[1][:rows_out * d_v * 2].view(torch.bfloat16).view(out.shape),
+                          res_d2[1][out_bytes:].view(torch.float32).view(lse.shape))]
+    res_h2 = [res_h, torch.empty_like(res_h).pin_memory()]
+    ev_in, ev_c, ev_out = ([torch.cuda.Event() for _ in range(KE)] for _ in range(3))
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    p0.record(s_in)
+    for k in range(KE):
+        i = k % 2
+        if k >= 2:
+            s_in.wait_event(ev_c[k - 2])     # input buffer i: step k - 2 has read it
+        with torch.cuda.stream(s_in):
+            in_d2[i].copy_(in_h, non_blocking=True)
+        ev_in[k].record(s_in)
+        stream.wait_event(ev_in[k])
+        if k >= 2:
+            stream.wait_event(ev_out[k - 2])  # result buffer i: step k - 2's result is out
+        with torch.cuda.stream(stream):
+            evict_l2()
+            step(*views2[i], *outs2[i])
+        ev_c[k].record(stream)
+        s_out.wait_event(ev_c[k])
+        with torch.cuda.stream(s_out):
+            res_h2[i].copy_(res_d2[i], non_blocking=True)
+        ev_out[k].record(s_out)
+    s_out.wait_event(ev_out[KE - 1])
+    p1.record(s_out)
+    torch.cuda.synchronize(dev)
+    e2e_pipe_ms = p0.elapsed_time(p1) / KE
+    if not (torch.equal(res_h2[0], res_h2[1]) if KE >= 2 else True):
+        raise SystemExit("the two result buffers of the pipelined e2e loop differ")
     err = binding.read_device_error(ws, stream)
     if err:
         raise SystemExit(f"device error flags after timing: {err}")
@@ -604,8 +647,9 @@ def main():
 
     t_step = statistics.mean(step_ms)
     t_kern = statistics.mean(kern_ms)
-    t_e2e = statistics.mean(e2e_ms)
-    t_step, t_kern, t_e2e = max_over_ranks([t_step, t_kern, t_e2e], pg, device=dev)
+    t_e2e_serial = statistics.mean(e2e_ms)
+    t_step, t_kern, t_e2e, t_e2e_serial = max_over_ranks([t_step, t_kern, e2e_pipe_ms, t_e2e_serial], pg,
+                                                         device=dev)
 
     hbm, tfl, peak_src = load_peaks()
     variant_kind = kernel_kind(inp)
@@ -636,7 +680,11 @@ def main():
             "roofline_frac_of_step": roof["roofline_us"] / (t_step * 1e3),
             "roofline": roof,
             "e2e": {"value": t_e2e * 1e3, "unit": UNIT,
-                    "h2d_bytes_per_step": int(in_h.numel()), "d2h_bytes_per_step": int(res_h.numel())},
+                    "h2d_bytes_per_step": int(in_h.numel()), "d2h_bytes_per_step": int(res_h.numel()),
+                    "schedule": "two buffer sets; step k+1's H2D and step k-1's D2H overlap step k on their "
+                                "own streams; per step = whole loop / steps",
+                    "serial_value": t_e2e_serial * 1e3,
+                    "serial_schedule": "H2D, the call, D2H on one stream, mean of per-step events"},
             "gpu_launches": K * launches_per_step, "timed_region_wall_s": t_wall,
             "kernel_timing": ("whole steps (cascade: several decode launches per step)" if args.cascade else
                               "second pass of K steps with events around the decode kernel"),

@@ -43,8 +43,12 @@ namespace {
 constexpr int NARROW_TOK = 96;  // tokens per tile
 constexpr int NMAXSEG = 32;
 constexpr int NSMX = 4;     // softmax warps
-constexpr int NGATHER = 3;  // gather warps (0, 2, 3)
-constexpr int NTHREADS = 32 * (4 + NSMX);
+// GW producer warps: 0, 2, 3 and, for gathered tiles, 8 .. GW + 4 (warps 4-7 are the softmax
+// warps: their lane quadrant is warp % 4)
+constexpr int BOX_WARPS = 3;
+constexpr int GATHER_WARPS = 5;
+template <int GW>
+constexpr int narrow_threads() { return 32 * (4 + NSMX + GW - 3); }
 constexpr float RESCALE_LOG2 = 8.f;
 constexpr int PF = 2;       // tiles ahead of the load that the producer prefetches into L2
 
@@ -118,8 +122,8 @@ __device__ __forceinline__ void store_half_row(uint32_t taddr, const uint32_t (&
     }
 }
 
-template <int TOK>
-__global__ void __launch_bounds__(NTHREADS, 1)
+template <int TOK, int GW>
+__global__ void __launch_bounds__(narrow_threads<GW>(), 1)
     gla_narrow_kernel(const __grid_constant__ CUtensorMap latmap, const __grid_constant__ CUtensorMap ropemap,
                       const LatentArgs a) {
     using C = NarrowCfg<TOK>;
@@ -147,7 +151,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
-            mbar_init(&full_bar[s], a.gather ? 32 * NGATHER : 1);  // gathered: one arrival per gather lane
+            mbar_init(&full_bar[s], a.gather ? 32 * GW : 1);  // gathered: one arrival per gather lane
             mbar_init(&empty_bar[s], 1);
         }
         mbar_init(&qfull_bar, 32 * NSMX);  // one cp.async arrival per softmax thread
@@ -178,7 +182,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // softmax thread geometry: quadrant qd, half of the row's scores, row slot in the quadrant
     const int qd = warp & 3;
     const int half = lane >> 4, rl = lane & 15;
-    const int n_row = (warp >= 4 && rl < rq) ? qd * rq + rl : R;
+    const bool smx_warp = warp >= 4 && warp < 8;
+    const int n_row = (smx_warp && rl < rq) ? qd * rq + rl : R;
     const bool row_ok = n_row < R;
     const bool warp_live = qd * rq < R;  // some row of this warp is real
     const int i_row = row_ok ? n_row / g : 0;
@@ -187,7 +192,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     // q rows of sequence b into shared memory (MMA row 16 qd + rl), this thread's half of the
     // row's 40 16-byte units; every softmax thread arrives on qfull once its copies landed
-    const uint64_t q_pol = warp >= 4 ? policy_evict_first() : 0;
+    const uint64_t q_pol = smx_warp ? policy_evict_first() : 0;
     auto load_q = [&](int b) {
         if (row_ok) {
             const __nv_bfloat16 *src = a.q + ((size_t)(b * a.L + i_row) * a.h_q + head) * C::DQK;
@@ -215,9 +220,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncthreads();
         const int nseg = nseg_sh;
 
-        if (warp == 0 || warp == 2 || warp == 3) {
+        if (warp == 0 || warp == 2 || warp == 3 || warp >= 8) {
             // ================================================================ producer(s)
-            const int gw = warp == 0 ? 0 : warp - 1;
+            const int gw = warp == 0 ? 0 : (warp < 4 ? warp - 1 : warp - 5);
             const uint64_t pol = policy_evict_first();
             const uint64_t pol_rope = policy_evict_normal();
             bool stop = false;
@@ -226,15 +231,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int T = clamp_len(__ldg(a.seqlens + sg.b), max_tokens, a.L, nullptr);
                 const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
                 if (a.gather) {
-                    // the gather warps split a tile's tokens k = gw, gw + 3, ..; lane i resolves the
+                    // the gather warps split a tile's tokens k = gw, gw + GW, ..; lane i resolves the
                     // cache row of the warp's i-th token (a tile ahead) and the warp copies each
                     // token's latent and rope rows into the box layout; every lane arrives on the
                     // stage barrier once its copies have landed
-                    static_assert(TOK <= 32 * NGATHER, "one token per gather lane");
+                    static_assert(TOK <= 32 * GW, "one token per gather lane");
                     const __nv_bfloat16 *lat = (const __nv_bfloat16 *)a.cache0 + (size_t)c * C::DC;
                     const __nv_bfloat16 *rope = (const __nv_bfloat16 *)a.cache1;
-                    const int nk = (TOK - gw + NGATHER - 1) / NGATHER;
-                    auto tok_of = [&](int t) { return min(t * TOK + gw + NGATHER * lane, T - 1); };
+                    const int nk = (TOK - gw + GW - 1) / GW;
+                    auto tok_of = [&](int t) { return min(t * TOK + gw + GW * lane, T - 1); };
                     int nxt = lane < nk ? __ldg(bt + tok_of(sg.t0) / a.page_size) : 0;
                     for (int t = sg.t0; t < sg.t1 && !stop; ++t) {
                         int pg = nxt;
@@ -256,7 +261,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0) {
                             const uint32_t st = smem_u32(stage_s + (size_t)stage * C::STAGE);
                             gather_tile<C::NV, 8>(st, C::CHUNK, lat, (size_t)a.h_c * C::DC, rope, 64,
-                                                  st + C::NV * C::CHUNK, myrow, gw, NGATHER, nk, lane, pol);
+                                                  st + C::NV * C::CHUNK, myrow, gw, GW, nk, lane, pol);
                             cp_async_arrive(&full_bar[stage]);
                         }
                         ++p_issued;
@@ -270,7 +275,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // tile's 5 nbox copies from one warp fell behind the stream
                 const int box_tok = a.box_tok;
                 const int nbox = TOK / box_tok;
-                const int kbox = gw + NGATHER * lane;  // this lane's box of every tile
+                const int kbox = gw + GW * lane;  // this lane's box of every tile
                 // block-table entries are read two tiles ahead of their use, so that their latency
                 // overlaps the stage waits; NO_BOX marks a box past T_b
                 constexpr int NO_BOX = -2147483647 - 1;
@@ -412,7 +417,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
             __syncwarp();
-        } else if (warp >= 4) {
+        } else if (smx_warp) {
             // ================================================================ softmax / epilogue
             const int st_id = threadIdx.x - 128;  // 0 .. 127
             bool ok = true;
@@ -590,12 +595,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-template <int TOK>
+template <int TOK, int GW>
 cudaError_t launch_t(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid, cudaStream_t st) {
-    auto k = gla_narrow_kernel<TOK>;
+    auto k = gla_narrow_kernel<TOK, GW>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)NarrowCfg<TOK>::SMEM);
     if (e != cudaSuccess) return e;
-    k<<<grid, NTHREADS, NarrowCfg<TOK>::SMEM, st>>>(lm, rm, a);
+    k<<<grid, narrow_threads<GW>(), NarrowCfg<TOK>::SMEM, st>>>(lm, rm, a);
     return cudaGetLastError();
 }
 
@@ -610,7 +615,10 @@ size_t narrow_smem_bytes() { return NarrowCfg<NARROW_TOK>::SMEM; }
 
 cudaError_t launch_gla_narrow(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid,
                               cudaStream_t st) {
-    return launch_t<NARROW_TOK>(lm, rm, a, grid, st);
+    // gathered tiles: more producer warps, as the copy-issue rate of three bounds the kernel; the
+    // box path keeps the smaller block (and its register bound)
+    return a.gather ? launch_t<NARROW_TOK, GATHER_WARPS>(lm, rm, a, grid, st)
+                    : launch_t<NARROW_TOK, BOX_WARPS>(lm, rm, a, grid, st);
 }
 
 }  // namespace kvd

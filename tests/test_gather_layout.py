@@ -108,7 +108,7 @@ def gather_tile(nch, rw, chunk_bytes, k0, kstep, nk, row_of):
 
 
 @pytest.mark.parametrize("nch,rw,tok", [(4, 8, 64), (2, 8, 64), (4, 4, 64), (4, 8, 96)])  # GLA d_c 256 (64- and
-@pytest.mark.parametrize("nwarps", [3, 5])                                                  # 96-token tiles), GTA
+@pytest.mark.parametrize("nwarps", [3, 5, 6])                                               # 96-token tiles), GTA
 def test_latent_gather_covers_the_box_layout(nch, rw, tok, nwarps):                          # prefix, MLA half
     if (tok + nwarps - 1) // nwarps > 32:
         pytest.skip("one token per gather lane")
