@@ -259,8 +259,9 @@ struct LatentPlan {
     int spread;  // rows per lane quadrant when the rows are spread (0: not spread)
     bool gather;
     bool narrow;  // at most 64 rows per latent head of width 256: the narrow kernel
+    bool m128;    // 65 to 128 rows per latent head of width 256: the 128-row kernel
     int tile;     // tokens per plan tile
-    int box_tok;  // narrow kernel, box path: tokens per TMA box
+    int box_tok;  // narrow and 128-row kernels, box path: tokens per TMA box
     int seg_cost; // plan: units a segment start costs, in tiles
     LatentShape shape;
     bool pair;
@@ -310,12 +311,13 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
     lp->box_tok = 0;
     lp->seg_cost = 0;
     lp->narrow = !lp->pair && p->d_c == 256 && R <= 64;
-    if (lp->narrow) {
-        // rows spread over the four lane quadrants, ceil(R / 4) each; the tile is cut into boxes
-        // of the largest size that divides both the tile and the page (at least 16 tokens), else
-        // gathered token by token
-        lp->spread = (int)((R + 3) / 4);
-        lp->tile = narrow_tile_tokens();
+    lp->m128 = !lp->pair && p->d_c == 256 && R > 64 && R <= 128;
+    if (lp->narrow || lp->m128) {
+        // narrow: rows spread over the four lane quadrants, ceil(R / 4) each; 128-row kernel: row
+        // n at TMEM lane n.  The tile is cut into boxes of the largest size that divides both the
+        // tile and the page (at least 16 tokens), else gathered token by token
+        lp->spread = lp->narrow ? (int)((R + 3) / 4) : 0;
+        lp->tile = lp->narrow ? narrow_tile_tokens() : m128_tile_tokens();
         int gcd = lp->tile, b2 = p->page_size;
         while (b2) {
             const int t = gcd % b2;
@@ -324,11 +326,11 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
         }
         lp->box_tok = gcd >= 16 ? gcd : 0;
         lp->gather = lp->box_tok == 0;
-        lp->seg_cost = narrow_seg_cost();
+        lp->seg_cost = lp->narrow ? narrow_seg_cost() : m128_seg_cost();
         lp->nstage = 0;
-        lp->smem = narrow_smem_bytes();
+        lp->smem = lp->narrow ? narrow_smem_bytes() : m128_smem_bytes();
     }
-    if (!lp->narrow) {
+    if (!lp->narrow && !lp->m128) {
         const size_t fixed = SMEM_PER_BLOCK - LATENT_STATIC_SMEM - 1024 - sh.q_bytes - sh.p_bytes;
         int nstage = (int)(fixed / sh.stage_bytes);
         if (nstage > MAX_STAGES) nstage = MAX_STAGES;
@@ -361,7 +363,7 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
     const int kch = d_qk / 64;
     const cuuint64_t tokens = (cuuint64_t)p->num_pages * p->page_size;
     CUtensorMap qm, lm, rm;
-    if (lp.narrow) {
+    if (lp.narrow || lp.m128) {
         memset(&qm, 0, sizeof(qm));  // q rows are copied by the kernel's softmax warps
         memset(&lm, 0, sizeof(lm));
         memset(&rm, 0, sizeof(rm));
@@ -468,6 +470,8 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
             return KVD_ERR_CUDA;
     } else if (lp.narrow) {
         if (launch_gla_narrow(lm, rm, a, lp.parts * lp.n_sub, st) != cudaSuccess) return KVD_ERR_CUDA;
+    } else if (lp.m128) {
+        if (launch_gla_m128(lm, rm, a, lp.parts * lp.n_sub, st) != cudaSuccess) return KVD_ERR_CUDA;
     } else if (launch_latent_decode(p->d_c, qm, lm, rm, a, lp.parts * lp.n_sub, lp.smem, st) != cudaSuccess) {
         return KVD_ERR_CUDA;
     }

@@ -96,6 +96,14 @@ size_t narrow_smem_bytes();
 cudaError_t launch_gla_narrow(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid,
                               cudaStream_t st);
 
+// GLA with 65 to 128 query rows per latent head (latent_m128.cu): 64-token tiles, M = 128 MMAs,
+// q in shared memory, two softmax warps per lane quadrant; no q tensor map.
+int m128_tile_tokens();
+int m128_seg_cost();
+size_t m128_smem_bytes();
+cudaError_t launch_gla_m128(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid,
+                            cudaStream_t st);
+
 // d_c = 512 (MLA): CTA pairs splitting the key dimension (latent_pair.cu).
 uint32_t mla_pair_fixed_smem();   // q half + the exchange buffer
 uint32_t mla_pair_stage_bytes();  // one 64-token tile half

@@ -1,0 +1,618 @@
+// GLA decode (absorbed form) for latent heads attended by 65 to 128 query rows: GLA-2 at
+// q_len 2 (64 heads per latent head), GLA-8 at q_len 5 to 8 (16 heads per latent head).
+//
+// "Hardware-Efficient Attention for Fast Decoding", section 3.3.2: h_c latent heads of width
+// d_c = 256 plus one shared RoPE key of width 64; query head h attends latent head
+// c = h / (h_q / h_c) with key [latent_c ++ rope] and value latent_c.  With 128 rows per latent
+// head the step sits at ~2 h_q FLOPs per byte, at the B200 ridge (Figure 15 of the paper: GLA
+// at q_len 2 on both roofs), so the tensor pipe and the HBM stream both have to run near their
+// rates and neither may wait for the softmax.
+//
+// Tensor-core shape.  One 128-row MMA covers every row of the latent head.  S = Q K^T is
+// M = 128, N = TOK = 64 tokens, K = 320: 16 MMAs with q's latent part read from tensor memory
+// and 4 with its rope part read from shared memory (an A operand of 128 rows re-read from
+// shared memory by every one of 20 small-N MMAs held the tensor pipe to the shared-memory
+// rate), and O += P V is M = 128, N = 256, K = 64 (4 MMAs, P read from tensor memory, V
+// MN-major straight from the latent tile).  Tensor memory: O in columns [0, 256), two S buffers
+// of 64 columns (P(j) written as bf16 pairs over the first 32 columns of S(j)), q's latent part
+// in [384, 512).  Shared memory: q's rope part (16 KB) and five 40 KB stages.
+//
+// One CTA owns one contiguous part of the (sequence, 64-token tile) stream and one latent head.
+// Roles:
+//   warps 0, 2, 3  producers: per tile the latent and rope rows of each page box by TMA (128 B
+//                  swizzle) into the ring, boxes spread over the three warps; block-table
+//                  entries one lane per box.  Pages that are not whole boxes are gathered token
+//                  by token with cp.async by the three warps.
+//   warp 1         MMA issuer (one thread).
+//   warps 4..11    softmax, one row per TMEM lane and two warps per lane quadrant: warp w
+//                  (w < 8) takes the first 32 scores of each row of quadrant w % 4, warp w + 4
+//                  the last 32.  The two agree on each row's running maximum by exchanging their
+//                  tile maxima through shared memory once per tile (and their row sums once per
+//                  segment), with one mbarrier per quadrant and bounded waits.  fp32 online
+//                  softmax in base 2 with a lazy rescale of O (each warp of the pair rescales
+//                  its 128 value columns).  They also write each segment's q rows (latent part
+//                  into tensor memory, rope part into shared memory with cp.async) and the
+//                  epilogue.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvd {
+
+namespace {
+
+constexpr int M128_TOK = 64;  // tokens per tile
+constexpr int NMAXSEG = 32;
+constexpr int NSMX = 8;       // softmax warps: two per lane quadrant
+constexpr int GW = 3;         // producer warps 0, 2, 3
+constexpr int NTHREADS = 32 * (4 + NSMX);
+constexpr float RESCALE_LOG2 = 8.f;
+constexpr int PF = 2;         // tiles ahead of the load that the producer prefetches into L2
+
+struct M128Cfg {
+    static constexpr int TOK = M128_TOK;
+    static constexpr int DC = 256;                     // latent width (value columns)
+    static constexpr int NV = DC / 64;                 // 64-wide latent chunks
+    static constexpr int KCH = NV + 1;                 // key chunks: latent, then rope
+    static constexpr int DQK = DC + 64;                // q row: latent part, then rope
+    static constexpr uint32_t Q_BYTES = 128 * 128;     // q's rope part: 128 MMA rows x 64 dims
+    static constexpr uint32_t CHUNK = TOK * 128;       // one 64-dim chunk of a tile
+    static constexpr uint32_t STAGE = KCH * CHUNK;     // 40 KB
+    static constexpr int NSTAGE = 5;
+    static constexpr uint32_t SMEM = 1024 + Q_BYTES + NSTAGE * STAGE;
+    static constexpr int NS = TOK / 2;                 // scores of a row held by one thread
+    static constexpr uint32_t S_COL = DC;              // S/P buffers after O
+    static constexpr uint32_t Q_COL = S_COL + 2 * TOK; // q's latent part: DC / 2 columns of bf16 pairs
+    static constexpr uint32_t TMEM_COLS = 512;
+    static_assert(Q_COL + DC / 2 == TMEM_COLS, "O, two S/P buffers and q's latent part");
+    static_assert(SMEM <= 221 * 1024, "shared memory (with the static part)");
+};
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    gla_m128_kernel(const __grid_constant__ CUtensorMap latmap, const __grid_constant__ CUtensorMap ropemap,
+                    const LatentArgs a) {
+    using C = M128Cfg;
+    constexpr int TOK = C::TOK;
+    constexpr int NST = C::NSTAGE;
+    constexpr int NS = C::NS;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ uint64_t full_bar[NST], empty_bar[NST];
+    __shared__ uint64_t qfull_bar, sfull_bar[2], pfull_bar[2], end_bar;
+    __shared__ uint64_t xbar[4][2];          // per lane quadrant: the pair's exchange, two buffers
+    __shared__ float xch_sh[2][2][128][2];   // [buffer][half][row][value]
+    __shared__ Seg segs[NMAXSEG];
+    __shared__ int nseg_sh, more_sh;
+    __shared__ volatile int abort_sh;
+    __shared__ uint32_t tmem_sh;
+
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *q_s = smem;
+    uint8_t *stage_s = smem + C::Q_BYTES;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int part = blockIdx.x / a.h_c, c = blockIdx.x % a.h_c;
+    const int g = a.h_q / a.h_c;
+    const int R = g * a.L;  // 64 < R <= 128
+    const int max_tokens = a.max_pages * a.page_size;
+    const uint64_t lim_ns = a.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(&full_bar[s], a.gather ? 32 * GW : 1);  // gathered: one arrival per gather lane
+            mbar_init(&empty_bar[s], 1);
+        }
+        // one cp.async arrival per softmax thread (q's rope rows) and one arrival per softmax warp
+        // (q's latent part written into tensor memory)
+        mbar_init(&qfull_bar, 32 * NSMX + NSMX);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sfull_bar[s], 1);
+            mbar_init(&pfull_bar[s], NSMX);  // one arrival per softmax warp
+        }
+        for (int q = 0; q < 4; ++q)
+            for (int s = 0; s < 2; ++s) mbar_init(&xbar[q][s], 2);  // the two warps of a quadrant
+        mbar_init(&end_bar, 1);
+        abort_sh = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&tmem_sh, C::TMEM_COLS);
+    if (warp == 0 && lane == 0 && !a.gather) {
+        tma_prefetch_desc(&latmap);
+        tma_prefetch_desc(&ropemap);
+    }
+    pdl_launch_dependents();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_sh;
+
+    // counters that persist across segment-list rounds
+    uint32_t p_issued = 0;                          // producer
+    uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;  // MMA issuer
+    uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0;  // softmax (x_x: pair exchanges)
+
+    // softmax thread geometry: row n = 32 qd + lane (MMA row = TMEM lane), score half `half`
+    const bool smx_warp = warp >= 4 && warp < 4 + NSMX;
+    const int qd = warp & 3;
+    const int half = smx_warp ? (warp - 4) >> 2 : 0;
+    const int n_row = smx_warp ? 32 * qd + lane : 0;
+    const bool row_ok = smx_warp && n_row < R;
+    const bool warp_live = 32 * qd < R;  // some row of this quadrant is real
+    const int i_row = row_ok ? n_row / g : 0;
+    const int head = row_ok ? c * g + n_row % g : 0;
+    const uint32_t s_lanes = (uint32_t)(qd * 32) << 16;
+
+    // q row n of sequence b: this thread's half of the latent part (128 dims, 64 columns of bf16
+    // pairs) into its TMEM lane, its half of the rope part (4 of 8 16-byte units) into shared
+    // memory (MMA row n).  Called by whole softmax warps once no score product reads q any more.
+    const uint64_t q_pol = smx_warp ? policy_evict_first() : 0;
+    auto load_q = [&](int b) {
+        const __nv_bfloat16 *src = a.q + ((size_t)(b * a.L + i_row) * a.h_q + head) * C::DQK;
+        if (row_ok) {
+            const uint32_t dst = smem_u32(q_s);
+#pragma unroll
+            for (int u = 4 * half; u < 4 * half + 4; ++u)
+                cp_async16(dst + sw128((uint32_t)n_row, (uint32_t)u), src + C::DC + u * 8, q_pol);
+        }
+        cp_async_arrive(&qfull_bar);
+        const uint4 *lat = (const uint4 *)(src + half * (C::DC / 2));
+#pragma unroll 1
+        for (int p16 = 0; p16 < 4; ++p16) {
+            uint32_t w[16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint4 v = row_ok ? __ldg(lat + p16 * 4 + k) : make_uint4(0, 0, 0, 0);
+                w[4 * k] = v.x;
+                w[4 * k + 1] = v.y;
+                w[4 * k + 2] = v.z;
+                w[4 * k + 3] = v.w;
+            }
+            tmem_st16u(tmem + s_lanes + C::Q_COL + half * (C::DC / 4) + p16 * 16, w);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qfull_bar);
+    };
+
+    // the pair of softmax warps of a quadrant swap two values per row: each writes its own, both
+    // arrive, each reads the other's.  Buffer x_x & 1 is written again two exchanges later, after
+    // the partner has passed the exchange in between and so has read it.  The exchange also
+    // orders the pair's tensor-memory accesses: what one warp read before it (its scores) is read
+    // before what the other writes after it (P over those columns).
+    auto exchange = [&](float v0, float v1, float &p0, float &p1) -> bool {
+        const uint32_t bf = x_x & 1;
+        xch_sh[bf][half][n_row][0] = v0;
+        xch_sh[bf][half][n_row][1] = v1;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xbar[qd][bf]);
+        if (!mbar_wait_warp(&xbar[qd][bf], (x_x >> 1) & 1, &abort_sh, a.err, lim_ns)) return false;
+        tc_fence_after();
+        p0 = xch_sh[bf][half ^ 1][n_row][0];
+        p1 = xch_sh[bf][half ^ 1][n_row][1];
+        ++x_x;
+        return true;
+    };
+
+    for (int skip = 0;; skip += NMAXSEG) {
+        if (warp == 0) {
+            int cnt = 0;
+            plan_walk(a.seqlens, a.B, TOK, a.seg_cost, max_tokens, a.L, part, a.parts, a.err, [&](const Seg &s) {
+                if (cnt >= skip && cnt < skip + NMAXSEG) segs[cnt - skip] = s;
+                ++cnt;
+            });
+            if (lane == 0) {
+                nseg_sh = cnt - skip < NMAXSEG ? (cnt - skip > 0 ? cnt - skip : 0) : NMAXSEG;
+                more_sh = cnt > skip + NMAXSEG;
+            }
+        }
+        __syncthreads();
+        const int nseg = nseg_sh;
+
+        if (warp == 0 || warp == 2 || warp == 3) {
+            // ================================================================ producers
+            const int gw = warp == 0 ? 0 : warp - 1;
+            const uint64_t pol = policy_evict_first();
+            const uint64_t pol_rope = policy_evict_normal();
+            bool stop = false;
+            for (int si = 0; si < nseg && !stop; ++si) {
+                const Seg sg = segs[si];
+                const int T = clamp_len(__ldg(a.seqlens + sg.b), max_tokens, a.L, nullptr);
+                const int32_t *bt = a.block_table + (size_t)sg.b * a.max_pages;
+                if (a.gather) {
+                    // the gather warps split a tile's tokens k = gw, gw + GW, ..; lane i resolves the
+                    // cache row of the warp's i-th token (a tile ahead) and the warp copies each
+                    // token's latent and rope rows into the box layout; every lane arrives on the
+                    // stage barrier once its copies have landed
+                    static_assert(TOK <= 32 * GW, "one token per gather lane");
+                    const __nv_bfloat16 *lat = (const __nv_bfloat16 *)a.cache0 + (size_t)c * C::DC;
+                    const __nv_bfloat16 *rope = (const __nv_bfloat16 *)a.cache1;
+                    const int nk = (TOK - gw + GW - 1) / GW;
+                    auto tok_of = [&](int t) { return min(t * TOK + gw + GW * lane, T - 1); };
+                    int nxt = lane < nk ? __ldg(bt + tok_of(sg.t0) / a.page_size) : 0;
+                    for (int t = sg.t0; t < sg.t1 && !stop; ++t) {
+                        int pg = nxt;
+                        if (t + 1 < sg.t1 && lane < nk) nxt = __ldg(bt + tok_of(t + 1) / a.page_size);
+                        const uint32_t stage = p_issued % NST;
+                        if (!mbar_wait_warp(&empty_bar[stage], ((p_issued / NST) & 1) ^ 1, &abort_sh, a.err,
+                                            lim_ns)) {
+                            stop = true;
+                            break;
+                        }
+                        int myrow = 0;
+                        if (lane < nk) {
+                            if (pg < 0 || pg >= a.num_pages) {
+                                set_error(a.err, DEVERR_BAD_PAGE);
+                                pg = 0;
+                            }
+                            myrow = pg * a.page_size + tok_of(t) % a.page_size;
+                        }
+                        if (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0) {
+                            const uint32_t st = smem_u32(stage_s + (size_t)stage * C::STAGE);
+                            gather_tile<C::NV, 8>(st, C::CHUNK, lat, (size_t)a.h_c * C::DC, rope, 64,
+                                                  st + C::NV * C::CHUNK, myrow, gw, GW, nk, lane, pol);
+                            cp_async_arrive(&full_bar[stage]);
+                        }
+                        ++p_issued;
+                    }
+                    continue;
+                }
+                // box path: a tile is nbox boxes of box_tok tokens, each inside one page; boxes
+                // that start at or past T are not loaded (their rows are masked and zeroed); box k
+                // is issued by warp k % 3, lane k / 3
+                const int box_tok = a.box_tok;
+                const int nbox = TOK / box_tok;
+                const int kbox = gw + GW * lane;  // this lane's box of every tile
+                // block-table entries are read two tiles ahead of their use; NO_BOX marks a box
+                // past T_b
+                constexpr int NO_BOX = -2147483647 - 1;
+                auto raw_entry = [&](int t) -> int {
+                    const int tok = t * TOK + kbox * box_tok;
+                    return (t < sg.t1 && kbox < nbox && tok < T) ? __ldg(bt + tok / a.page_size) : NO_BOX;
+                };
+                auto cache_row = [&](int raw, int t) -> int {  // cache row of this lane's box of tile t
+                    if (raw == NO_BOX) return -1;
+                    if (raw < 0 || raw >= a.num_pages) {
+                        set_error(a.err, DEVERR_BAD_PAGE);
+                        raw = 0;
+                    }
+                    return raw * a.page_size + (t * TOK + kbox * box_tok) % a.page_size;
+                };
+                // warp 0 of the first latent head's CTA brings the pages of tile t + PF into L2
+                // when it loads tile t (whole pages, every latent head and the rope rows, one
+                // untiled bulk prefetch each)
+                const bool pf_warp = warp == 0 && c == 0;
+                const size_t lat_page = (size_t)a.page_size * a.h_c * C::DC * 2, rope_page = (size_t)a.page_size * 128;
+                int pf_next_page = -1;  // logical page index prefetched next (pages already done: below)
+                auto raw_page = [&](int t) -> int {  // lane j: the j-th page of tile t
+                    const int p0 = t * TOK / a.page_size, p1 = (min(t * TOK + TOK, T) - 1) / a.page_size;
+                    return (pf_warp && t < sg.t1 && p0 + lane <= p1) ? __ldg(bt + p0 + lane) : NO_BOX;
+                };
+                int raw_ld = raw_entry(sg.t0), raw_nx = raw_entry(sg.t0 + 1);
+                int raw_pf = raw_page(sg.t0 + PF), raw_pf_nx = raw_page(sg.t0 + PF + 1);
+                for (int t = sg.t0; t < sg.t1 && !stop; ++t) {
+                    const int row = cache_row(raw_ld, t);
+                    const int pf = raw_pf;
+                    raw_ld = raw_nx;
+                    raw_nx = raw_entry(t + 2);
+                    raw_pf = raw_pf_nx;
+                    raw_pf_nx = raw_page(t + PF + 2);
+                    const uint32_t stage = p_issued % NST;
+                    if (!mbar_wait_warp(&empty_bar[stage], ((p_issued / NST) & 1) ^ 1, &abort_sh, a.err, lim_ns)) {
+                        stop = true;
+                        break;
+                    }
+                    if (warp == 0 && lane == 0) {
+                        const int nb = min(nbox, (T - t * TOK + box_tok - 1) / box_tok);
+                        mbar_arrive_expect_tx(&full_bar[stage], (uint32_t)(nb * box_tok * C::DQK * 2));
+                    }
+                    if (row >= 0 && (!(a.debug_flags & DEBUG_SKIP_FIRST_LOAD) || p_issued != 0)) {
+                        uint8_t *st = stage_s + (size_t)stage * C::STAGE + (size_t)kbox * box_tok * 128;
+                        if (box_tok == TOK) {  // one box of all four latent chunks
+                            tma_load_3d(st, &latmap, &full_bar[stage], 0, row, c * C::NV, pol);
+                        } else {
+#pragma unroll
+                            for (int ch = 0; ch < C::NV; ++ch)
+                                tma_load_3d(st + ch * C::CHUNK, &latmap, &full_bar[stage], 0, row, c * C::NV + ch, pol);
+                        }
+                        // the rope rows are read by every latent head's CTA: no evict-first hint
+                        tma_load_2d(st + C::NV * C::CHUNK, &ropemap, &full_bar[stage], 0, row, pol_rope);
+                    }
+                    if (pf_warp && t + PF < sg.t1) {
+                        const int p0 = (t + PF) * TOK / a.page_size;
+                        const int p1 = (min((t + PF) * TOK + TOK, T) - 1) / a.page_size;
+                        const int pg = pf < 0 || pf >= a.num_pages ? 0 : pf;
+                        if (p0 + lane <= p1 && p0 + lane >= pf_next_page) {
+                            bulk_prefetch_l2((const uint8_t *)a.cache0 + (size_t)pg * lat_page, (uint32_t)lat_page);
+                            bulk_prefetch_l2((const uint8_t *)a.cache1 + (size_t)pg * rope_page, (uint32_t)rope_page);
+                        }
+                        pf_next_page = p1 + 1;
+                    }
+                    ++p_issued;
+                }
+            }
+            if (stop) {
+                // let every copy already issued land before the CTA can exit
+                volatile int never = 0;
+                if (a.gather) {
+                    asm volatile("cp.async.wait_all;" ::: "memory");
+                } else {
+                    const uint32_t lo = p_issued > (uint32_t)NST ? p_issued - NST : 0;
+                    for (uint32_t k = lo; k < p_issued; ++k)
+                        mbar_wait_warp(&full_bar[k % NST], (k / NST) & 1, &never, nullptr, lim_ns);
+                }
+            }
+        } else if (warp == 1) {
+            // ================================================================ MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t idesc_s = umma_idesc_bf16(128, TOK, false, false);
+                constexpr uint32_t idesc_pv = umma_idesc_bf16(128, C::DC, false, true);
+                const uint32_t st0 = smem_u32(stage_s);
+                const uint64_t dq0 = umma_desc(smem_u32(q_s), 16, 1024, 2);
+                bool ok = true;
+                auto issue_s = [&](uint32_t gt) -> bool {
+                    const uint32_t stage = gt % NST;
+                    if (!mbar_wait_one(&full_bar[stage], (gt / NST) & 1, &abort_sh, a.err, lim_ns)) return false;
+                    tc_fence_after();
+                    if (a.gather) fence_proxy_async();  // rows written by cp.async, read by the tensor core
+                    // S(j) goes into buffer j & 1, over P(j - 2): the MMAs of one thread run in issue
+                    // order, so this product, issued after the P.V product of tile j - 2, cannot
+                    // overwrite that P before it is read
+                    const uint32_t d = tmem + C::S_COL + (m_s & 1) * TOK;
+                    const uint64_t dk0 = umma_desc(st0 + stage * C::STAGE, 16, 1024, 2);
+#pragma unroll
+                    for (int kc = 0; kc < C::NV; ++kc)  // latent chunks: q from tensor memory
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16_ts(d, tmem + C::Q_COL + kc * 32 + kk * 8,
+                                         dk0 + (uint64_t)((kc * C::CHUNK + kk * 32) >> 4), idesc_s, (kc | kk) != 0);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)  // rope chunk: q from shared memory
+                        umma_bf16(d, dq0 + (uint64_t)((kk * 32) >> 4),
+                                  dk0 + (uint64_t)((C::NV * C::CHUNK + kk * 32) >> 4), idesc_s, 1u);
+                    umma_commit(&sfull_bar[m_s & 1]);
+                    ++m_s;
+                    return true;
+                };
+                for (int si = 0; si < nseg && ok; ++si) {
+                    const int n = segs[si].t1 - segs[si].t0;
+                    if (!mbar_wait_one(&qfull_bar, m_q & 1, &abort_sh, a.err, lim_ns)) break;
+                    ++m_q;
+                    tc_fence_after();
+                    fence_proxy_async();  // q's rope rows written by cp.async
+                    if (!issue_s(m_tile)) break;
+                    for (int j = 0; j < n; ++j) {
+                        if (j + 1 < n && !issue_s(m_tile + j + 1)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t pb = m_pv & 1;
+                        if (!mbar_wait_one(&pfull_bar[pb], (m_pv >> 1) & 1, &abort_sh, a.err, lim_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t stage = (m_tile + j) % NST;
+                        const uint64_t dv0 = umma_desc(st0 + stage * C::STAGE, C::CHUNK, 1024, 2);
+                        const uint32_t pa = tmem + C::S_COL + pb * TOK;  // P(j) over S(j): bf16 pairs
+#pragma unroll
+                        for (int kk = 0; kk < TOK / 16; ++kk)
+                            umma_bf16_ts(tmem, pa + kk * 8, dv0 + (uint64_t)(kk * 128), idesc_pv,
+                                         (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&empty_bar[stage]);  // the stage is free and P.V j is done
+                        ++m_pv;
+                    }
+                    m_tile += n;
+                }
+            }
+            __syncwarp();
+        } else if (smx_warp) {
+            // ================================================================ softmax / epilogue
+            const int st_id = threadIdx.x - 128;  // 0 .. 255
+            bool ok = true;
+            // wait until P.V number k has completed (O settled): the commit that frees tile k's
+            // stage.  P(k) needed S(k), issued after P.V k - 2, so every earlier P.V is complete
+            // and the barrier is at most one phase short of the one waited for.
+            auto wait_pv = [&](uint32_t k) -> bool {
+                return mbar_wait_warp(&empty_bar[k % NST], (k / NST) & 1, &abort_sh, a.err, lim_ns);
+            };
+            bool q_ready = false;  // this segment's q rows are already on their way
+            for (int si = 0; si < nseg && ok; ++si) {
+                const Seg sg = segs[si];
+                const int b = sg.b;
+                const int T = clamp_len(__ldg(a.seqlens + b), max_tokens, a.L, nullptr);
+                const int lim = row_ok ? T - a.L + i_row : -1;  // causal: row (i, h) sees t <= T - L + i
+                const int lim_all = T - a.L;                     // visible to every row
+                if (!q_ready) load_q(b);  // the q buffer is free: the previous segment's scores are done
+                q_ready = false;
+                // l: sum of the fp32 P (gives lse); lq: sum of the bf16-rounded P the product uses;
+                // both over this warp's half of the row until the segment's end
+                float m_ref = -INFINITY, l = 0.f, lq = 0.f;
+                for (int tile = sg.t0; tile < sg.t1; ++tile) {
+                    const int tok0 = tile * TOK;
+                    const uint32_t sb = x_s & 1;
+                    if (!mbar_wait_warp(&sfull_bar[sb], (x_s >> 1) & 1, &abort_sh, a.err, lim_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    ++x_s;
+                    // the segment's last score product is done: q may be overwritten by the next
+                    // segment's rows while this tile and the epilogue run
+                    if (tile + 1 == sg.t1 && si + 1 < nseg) {
+                        load_q(segs[si + 1].b);
+                        q_ready = true;
+                    }
+                    float s[NS];
+                    const int tok0_t = tok0 + half * NS;  // this thread's first token
+                    float mx = -INFINITY;
+                    const bool full = tok0 + TOK - 1 <= lim_all;  // nothing masked in the tile
+                    if (warp_live) {
+                        tmem_ld32(tmem + s_lanes + C::S_COL + sb * TOK + half * NS, s);
+                        mx = tile_max(s, full, tok0_t, lim, a.scale_log2);
+                        if (!row_ok) mx = -INFINITY;
+                    }
+                    float mx_p, unused;
+                    if (!exchange(mx, 0.f, mx_p, unused)) {
+                        ok = false;
+                        break;
+                    }
+                    mx = fmaxf(mx, mx_p);  // the same value in both warps of the pair
+                    float alpha = 1.f;
+                    bool need = false;
+                    if (mx != -INFINITY) {
+                        if (m_ref == -INFINITY) {
+                            m_ref = mx;  // nothing visible before: O and the sums hold zeros
+                        } else if (mx > m_ref + RESCALE_LOG2) {
+                            alpha = ex2(m_ref - mx);
+                            need = true;
+                            m_ref = mx;
+                        }
+                    }
+                    if (__any_sync(0xffffffffu, need)) {
+                        // O is settled once the previous P.V (and so every earlier one) is done
+                        if (x_pv > 0 && !wait_pv(x_pv - 1)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        l *= alpha;
+                        lq *= alpha;
+                        // warp half h rescales O columns [128 h, 128 h + 128) of its rows
+#pragma unroll 1
+                        for (int ch = 0; ch < C::DC / 64; ++ch) {
+                            float o[32];
+                            tmem_ld32(tmem + s_lanes + half * (C::DC / 2) + ch * 32, o);
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) o[k] *= alpha;
+                            tmem_st32(tmem + s_lanes + half * (C::DC / 2) + ch * 32, o);
+                        }
+                        tmem_st_wait();
+                    }
+                    if (warp_live) l += tile_exp(s, full, tok0_t, lim, a.scale_log2, m_ref);
+
+                    // tokens past T_b in this tile hold garbage or were never loaded: zero their
+                    // value rows (P is 0 there, but 0 * NaN would still poison the product)
+                    const uint32_t stage = x_tile % NST;
+                    if (tok0 + TOK > T) {
+                        const int k0 = max(T - tok0, 0);
+                        uint8_t *v0 = stage_s + (size_t)stage * C::STAGE;
+                        const int units = (TOK - k0) * C::NV * 8;  // 16-byte units: rows x chunks x 8
+                        for (int u = st_id; u < units; u += 32 * NSMX) {
+                            const int row = k0 + u / (C::NV * 8), ch = (u / 8) % C::NV, k = u & 7;
+                            *(uint4 *)(v0 + ch * C::CHUNK + row * 128 + k * 16) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    // P (bf16 pairs) over S in the same buffer: this warp's 32 tokens are columns
+                    // [16 h, 16 h + 16) of it (the other warp of the pair has read those scores:
+                    // both passed the exchange after reading theirs)
+                    if (warp_live) {
+                        uint32_t w[NS / 2];
+                        float sum = 0.f, sum2 = 0.f;
+#pragma unroll
+                        for (int k = 0; k < NS / 2; ++k) {
+                            w[k] = pack_bf16(s[2 * k], s[2 * k + 1]);
+                            sum += bf16_lo(w[k]);
+                            sum2 += bf16_hi(w[k]);
+                        }
+                        tmem_st16u(tmem + s_lanes + C::S_COL + sb * TOK + half * (NS / 2), w);
+                        tmem_st_wait();
+                        lq += sum + sum2;
+                    }
+                    if (tok0 + TOK > T) fence_proxy_async();  // the zeroed value rows above
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pfull_bar[x_pv & 1]);
+                    ++x_pv;
+                    ++x_tile;
+                }
+                if (!ok) break;
+
+                // ---- epilogue: O is final once the last P.V completes
+                if (!wait_pv(x_pv - 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                float l_p, lq_p;  // the other half's sums (added in the same order in both warps)
+                if (!exchange(l, lq, l_p, lq_p)) {
+                    ok = false;
+                    break;
+                }
+                l = half == 0 ? l + l_p : l_p + l;
+                lq = half == 0 ? lq + lq_p : lq_p + lq;
+                const float inv = lq > 0.f ? 1.f / lq : 0.f;
+                const float lse_v = l > 0.f ? (m_ref + lg2(l)) * 0.69314718055994530942f : -INFINITY;
+                const size_t rows_b = (size_t)a.L * a.h_q;
+                const size_t r_out = (size_t)i_row * a.h_q + head;
+                if (warp_live) {
+#pragma unroll 1
+                    for (int ch = 0; ch < C::DC / 64; ++ch) {
+                        float o[32];
+                        tmem_ld32(tmem + s_lanes + half * (C::DC / 2) + ch * 32, o);
+                        if (!row_ok) continue;
+                        const int col = half * (C::DC / 2) + ch * 32;
+                        if (sg.nsplit == 1) {
+                            uint4 *op = (uint4 *)(a.out + ((size_t)b * rows_b + r_out) * C::DC + col);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                op[k] = make_uint4(pack_bf16(o[8 * k] * inv, o[8 * k + 1] * inv),
+                                                   pack_bf16(o[8 * k + 2] * inv, o[8 * k + 3] * inv),
+                                                   pack_bf16(o[8 * k + 4] * inv, o[8 * k + 5] * inv),
+                                                   pack_bf16(o[8 * k + 6] * inv, o[8 * k + 7] * inv));
+                        } else {
+                            float4 *op = (float4 *)(a.ws_o + ((size_t)sg.slot * rows_b + r_out) * C::DC + col);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                op[k] = make_float4(o[4 * k] * inv, o[4 * k + 1] * inv, o[4 * k + 2] * inv,
+                                                    o[4 * k + 3] * inv);
+                        }
+                    }
+                }
+                if (row_ok && half == 0) {
+                    if (sg.nsplit == 1)
+                        a.lse[(size_t)b * rows_b + r_out] = lse_v;
+                    else
+                        a.ws_lse[(size_t)sg.slot * rows_b + r_out] = lse_v;
+                }
+                tc_fence_before();
+            }
+            if (!ok) asm volatile("cp.async.wait_all;" ::: "memory");  // q copies in flight
+        }
+        __syncthreads();
+        if (!more_sh || abort_sh) break;
+        __syncthreads();
+    }
+
+    // every MMA issued by this CTA has completed before tensor memory is released
+    if (warp == 1 && lane == 0) {
+        volatile int never = 0;
+        umma_commit(&end_bar);
+        mbar_wait_one(&end_bar, 0, &never, nullptr, lim_ns);
+    }
+    if (smx_warp) asm volatile("cp.async.wait_all;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace
+
+int m128_tile_tokens() { return M128_TOK; }
+// A segment start costs the CTA a few µs (its q rows, the ring refilling, the epilogue of the
+// segment before it) against ~1 µs per 64-token tile at the HBM rate.
+int m128_seg_cost() { return 4; }
+size_t m128_smem_bytes() { return M128Cfg::SMEM; }
+
+cudaError_t launch_gla_m128(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid,
+                            cudaStream_t st) {
+    auto k = gla_m128_kernel;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)M128Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    k<<<grid, NTHREADS, M128Cfg::SMEM, st>>>(lm, rm, a);
+    return cudaGetLastError();
+}
+
+}  // namespace kvd

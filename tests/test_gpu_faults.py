@@ -27,6 +27,8 @@ CASES = {
                  scale=0.07),
     "gla2_q1": dict(variant="gla", B=2, L=1, h_q=128, h_kv=2, d=256, d_r=64, page_size=64, seqlens=[300, 90],
                     scale=0.07),
+    "gla2_q4": dict(variant="gla", B=2, L=4, h_q=128, h_kv=2, d=256, d_r=64, page_size=64, seqlens=[300, 90],
+                    scale=0.07),
     "mla": dict(variant="gla", B=2, L=1, h_q=128, h_kv=1, d=512, d_r=64, page_size=64, seqlens=[200, 90],
                 scale=0.07, latent_scale=0.1),
 }

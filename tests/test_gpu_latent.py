@@ -241,6 +241,72 @@ def test_latent_page_permutation_bit_identical(cuda_device):
     assert torch.equal(lse1, lse2)
 
 
+# ----------------------------------------------------------------------------- 65 to 128 rows per latent head
+# GLA-2 at q_len 2 and GLA-8 at q_len 5 to 8 run on the 128-row kernel (64-token tiles, M = 128,
+# two softmax warps per lane quadrant that exchange their row maxima every tile).
+@pytest.mark.parametrize("num_parts", [1, 3, 50, 148])
+def test_m128_forced_splits(cuda_device, num_parts):
+    inp = small(2, 256, B=5, L=2, seqlens=("uniform", 16, 1500), seed=311 + num_parts)
+    check(inp, num_parts=num_parts, what=f"GLA-2 L=2 parts={num_parts}")
+
+
+def test_m128_tile_boundaries(cuda_device):
+    sl = [2, 3, 31, 32, 63, 64, 65, 127, 128, 129, 300]
+    inp = small(2, 256, B=len(sl), L=2, seqlens=sl, seed=323)
+    for parts in (0, 1, 4, 64):
+        # stress bound: the two- and three-token sequences have rows that see one or two tokens
+        check(inp, num_parts=parts, what=f"GLA-2 L=2 tile boundaries parts={parts}", stress=True)
+
+
+@pytest.mark.parametrize("S", [1, 8, 16, 32, 48, 64, 128])
+def test_m128_page_sizes(cuda_device, S):
+    """Boxes of 16, 32 and 64 tokens (48: gcd 16), one box of the whole tile, and pages of 1 and 8
+    tokens gathered token by token."""
+    inp = small(2, 256, B=4, L=2, page_size=S, seqlens=("uniform", 30, 700), seed=329 + S)
+    check(inp, num_parts=5, what=f"GLA-2 L=2 S={S}")
+
+
+@pytest.mark.parametrize("h_c,h_q,L", [(8, 128, 5), (8, 128, 8), (4, 128, 3), (2, 128, 2)])
+def test_m128_row_counts(cuda_device, h_c, h_q, L):
+    """R = 80, 128, 96 and 128 rows: the last lane quadrants partly or wholly without rows."""
+    inp = small(h_c, 256, h_q=h_q, L=L, seqlens=("uniform", L + 8, 500), seed=337 + h_c + L)
+    check(inp, num_parts=3, what=f"h_c={h_c} h_q={h_q} L={L}")
+
+
+def test_m128_peaky_softmax(cuda_device):
+    inp = small(2, 256, L=2, seqlens=("uniform", 16, 2000), seed=347)
+    inp.scale *= 8
+    check(inp, num_parts=9)
+
+
+def test_m128_empty_sequences(cuda_device):
+    import torch
+    inp = small(2, 256, B=6, L=2, seqlens=[0, 70, 0, 5, 300, 0], seed=349)
+    d = gu.to_dev(inp)
+    out, lse = _nan_outputs(inp)
+    _gla_call(d, inp, out, lse, 3, torch.zeros(1 << 24, dtype=torch.uint8, device="cuda"))
+    o, l = gu.to_np(out, lse)
+    assert np.all(o[[0, 2, 5]] == 0) and np.all(np.isneginf(l[[0, 2, 5]]))
+    ref_o, ref_l, _ = orc.decode_inputs(inp)
+    gu.assert_close(o, l, ref_o, ref_l)
+
+
+def test_m128_page_permutation_bit_identical(cuda_device):
+    import torch
+    inp = small(2, 256, B=4, L=2, seqlens=("uniform", 2, 800), seed=353)
+    out1, lse1 = gu.run_gpu(inp)
+    perm = np.random.default_rng(5).permutation(inp.num_pages)
+    inv = np.argsort(perm)
+    for k in inp.caches:
+        inp.caches[k] = np.ascontiguousarray(inp.caches[k][inv])
+    bt = inp.block_table.copy()
+    bt[bt >= 0] = perm[bt[bt >= 0]]
+    inp.block_table = bt
+    out2, lse2 = gu.run_gpu(inp)
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(lse1, lse2)
+
+
 # ----------------------------------------------------------------------------- full workloads (sampled)
 def check_full(inp, b_sample, what):
     """A sample of sequences (always including the longest) against the oracle, plus every
