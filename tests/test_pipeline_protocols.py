@@ -1,7 +1,8 @@
 """Barrier protocols of the decode kernels, modelled on the CPU.
 
 Every warp role of the GQA/GTA kernel (group_decode.cu: box loads or gathered tiles), of the
-GLA kernel (latent_decode.cu) and of the MLA CTA-pair kernel (latent_pair.cu) is a coroutine that waits on and arrives at its mbarriers in the order the
+GLA kernels (latent_decode.cu, latent_narrow.cu, latent_m128.cu) and of the MLA CTA-pair kernel
+(latent_pair.cu) is a coroutine that waits on and arrives at its mbarriers in the order the
 kernel does; TMA copies, bulk copies to the peer CTA and tcgen05.commit arrivals complete later,
 in random order.  Random schedules over several segment patterns and stage counts must all
 finish (no stall), and no wait may find its barrier two or more phases past the phase it waits
@@ -269,6 +270,107 @@ def test_model_detects_a_missing_arrival():
         return schedule(gens, events, rnd, limit=20000)
 
     assert short(0, (3,), 2) == "stuck"
+
+
+def q_in_cta_model(seed, segs, nstage, pair, skip_exchange=False):
+    """gla_narrow_kernel (pair=False: four softmax warps) and gla_m128_kernel (pair=True: eight,
+    two per TMEM lane quadrant).  The softmax warps write each segment's q themselves: for the
+    first segment at its start, for every later one as soon as the previous segment's last score
+    product is done; their copies land later (an event) and, with `pair`, each warp also arrives
+    once its tensor-memory writes are out.  The MMA warp waits for q before a segment's first
+    score product.  With `pair` the two warps of a quadrant exchange their row maxima every tile
+    and their row sums at each segment end through two mbarriers of two arrivals, used
+    alternately."""
+    rnd = random.Random(seed)
+    events = []
+    nsmx = 8 if pair else 4
+    c = {"full": [Bar(f"full{s}", 1) for s in range(nstage)],
+         "empty": [Bar(f"empty{s}", 1) for s in range(nstage)],
+         "sfull": [Bar(f"sfull{s}", 1) for s in range(2)],
+         "pfull": [Bar(f"pfull{s}", nsmx) for s in range(2)],
+         "qfull": Bar("qfull", 2 * nsmx if pair else nsmx)}
+    xbar = [[Bar(f"x{q}{b}", 2) for b in range(2)] for q in range(4)]
+
+    def mma():
+        t = 0
+        for si, n in enumerate(segs):
+            yield from wait(lambda: c["qfull"].ready(si))
+
+            def issue_s(gt):
+                yield from wait(lambda: c["full"][gt % nstage].ready(gt // nstage))
+                events.append(lambda: c["sfull"][gt % 2].arrive())
+
+            yield from issue_s(t)
+            for j in range(n):
+                if j + 1 < n:
+                    yield from issue_s(t + j + 1)
+                yield from wait(lambda: c["pfull"][(t + j) % 2].ready((t + j) // 2))
+                st = (t + j) % nstage
+                events.append(lambda st=st: c["empty"][st].arrive())
+            t += n
+
+    def prod():
+        it = 0
+        for n in segs:
+            for _ in range(n):
+                st = it % nstage
+                yield from wait(lambda: it < nstage or c["empty"][st].ready(it // nstage - 1))
+                c["full"][st].expect_tx(1)
+                events.append(lambda st=st: c["full"][st].complete_tx(1))
+                it += 1
+
+    def softmax(w):
+        q = w % 4
+        x = 0
+        xx = [0]
+
+        def load_q():
+            events.append(lambda: c["qfull"].arrive())  # the copies land
+            if pair:
+                c["qfull"].arrive()  # the warp's tensor-memory writes are out
+
+        def exchange():
+            if skip_exchange and w == 4 and xx[0] == 1:
+                return
+            b = xx[0] % 2
+            xbar[q][b].arrive()
+            k = xx[0] // 2
+            yield from wait(lambda: xbar[q][b].ready(k))
+            xx[0] += 1
+
+        load_q()
+        for si, n in enumerate(segs):
+            for j in range(n):
+                yield from wait(lambda: c["sfull"][x % 2].ready(x // 2))
+                if j == n - 1 and si + 1 < len(segs):
+                    load_q()
+                if pair:
+                    yield from exchange() or ()
+                if x > 0 and rnd.random() < 0.3:  # lazy rescale: O settled after P.V(x - 1)
+                    yield from wait(lambda: c["empty"][(x - 1) % nstage].ready((x - 1) // nstage))
+                c["pfull"][x % 2].arrive()
+                x += 1
+            yield from wait(lambda: c["empty"][(x - 1) % nstage].ready((x - 1) // nstage))  # epilogue
+            if pair:
+                yield from exchange() or ()
+
+    gens = [prod(), mma()] + [softmax(w) for w in range(nsmx)]
+    return schedule(gens, events, rnd, limit=60000 if skip_exchange else 300000)
+
+
+@pytest.mark.parametrize("pair", [False, True], ids=["narrow", "m128"])
+@pytest.mark.parametrize("segs", SEGS)
+@pytest.mark.parametrize("nstage", [3, 5])
+def test_q_in_cta_protocols_finish_without_parity_aliasing(pair, segs, nstage):
+    ALIAS.clear()
+    for seed in range(25):
+        assert q_in_cta_model(seed, segs, nstage, pair) == "ok", seed
+    assert not ALIAS, ALIAS[:5]
+
+
+def test_pair_exchange_model_detects_a_skipped_exchange():
+    """One warp of a pair that skips an exchange leaves its partner waiting: the model stalls."""
+    assert q_in_cta_model(0, (3, 2), 3, True, skip_exchange=True) == "stuck"
 
 
 def mla_exchange_abort_model(seed, ntiles, abort_cta, abort_tiles, drain=True):
