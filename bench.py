@@ -44,12 +44,11 @@ UNIT = "us/step"
 FALLBACK_HBM_GBS, FALLBACK_TFLOPS = 6650.0, 1590.0
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB L2
 KERNEL_SOURCES = {"group": ["kv_cache_paged_b200/csrc/group_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"],
-                  "latent": ["kv_cache_paged_b200/csrc/latent_decode.cu", "kv_cache_paged_b200/csrc/common.cuh"],
                   "narrow": ["kv_cache_paged_b200/csrc/latent_narrow.cu", "kv_cache_paged_b200/csrc/common.cuh"],
                   "m128": ["kv_cache_paged_b200/csrc/latent_m128.cu", "kv_cache_paged_b200/csrc/common.cuh"],
                   "pair": ["kv_cache_paged_b200/csrc/latent_pair.cu", "kv_cache_paged_b200/csrc/common.cuh"],
                   "append": ["kv_cache_paged_b200/csrc/append.cu", "kv_cache_paged_b200/csrc/common.cuh"]}
-KERNEL_NAMES = {"group": "group_decode_kernel", "latent": "latent_decode_kernel", "narrow": "gla_narrow_kernel",
+KERNEL_NAMES = {"group": "group_decode_kernel", "narrow": "gla_narrow_kernel",
                 "m128": "gla_m128_kernel",
                 "pair": "mla_pair_kernel"}
 
@@ -60,10 +59,7 @@ def kernel_kind(inp):
         return "group"
     if inp.d == 512:
         return "pair"
-    rows = (inp.h_q // inp.h_kv) * inp.L  # query rows per latent head
-    if inp.d == 256 and rows <= 64:
-        return "narrow"
-    return "m128" if inp.d == 256 and rows <= 128 else "latent"
+    return "narrow" if (inp.h_q // inp.h_kv) * inp.L <= 64 else "m128"  # query rows per latent head
 
 
 def describe(inp):

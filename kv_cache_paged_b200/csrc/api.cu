@@ -259,7 +259,7 @@ struct LatentPlan {
     int spread;  // rows per lane quadrant when the rows are spread (0: not spread)
     bool gather;
     bool narrow;  // at most 64 rows per latent head of width 256: the narrow kernel
-    bool m128;    // 65 to 128 rows per latent head of width 256: the 128-row kernel
+    bool m128;    // more rows per latent head of width 256: the 128-row kernel, one CTA per 128 rows
     int tile;     // tokens per plan tile
     int box_tok;  // narrow and 128-row kernels, box path: tokens per TMA box
     int seg_cost; // plan: units a segment start costs, in tiles
@@ -311,11 +311,12 @@ int plan_latent(const kvd_gla_params *p, LatentPlan *lp) {
     lp->box_tok = 0;
     lp->seg_cost = 0;
     lp->narrow = !lp->pair && p->d_c == 256 && R <= 64;
-    lp->m128 = !lp->pair && p->d_c == 256 && R > 64 && R <= 128;
+    lp->m128 = !lp->pair && p->d_c == 256 && R > 64;
     if (lp->narrow || lp->m128) {
         // narrow: rows spread over the four lane quadrants, ceil(R / 4) each; 128-row kernel: row
-        // n at TMEM lane n.  The tile is cut into boxes of the largest size that divides both the
-        // tile and the page (at least 16 tokens), else gathered token by token
+        // 128 k + n at TMEM lane n of the k-th CTA of a latent head.  The tile is cut into boxes of
+        // the largest size that divides both the tile and the page (at least 16 tokens), else
+        // gathered token by token
         lp->spread = lp->narrow ? (int)((R + 3) / 4) : 0;
         lp->tile = lp->narrow ? narrow_tile_tokens() : m128_tile_tokens();
         int gcd = lp->tile, b2 = p->page_size;
@@ -472,8 +473,8 @@ int run_latent(const kvd_gla_params *p, void *ws, size_t ws_bytes, cudaStream_t 
         if (launch_gla_narrow(lm, rm, a, lp.parts * lp.n_sub, st) != cudaSuccess) return KVD_ERR_CUDA;
     } else if (lp.m128) {
         if (launch_gla_m128(lm, rm, a, lp.parts * lp.n_sub, st) != cudaSuccess) return KVD_ERR_CUDA;
-    } else if (launch_latent_decode(p->d_c, qm, lm, rm, a, lp.parts * lp.n_sub, lp.smem, st) != cudaSuccess) {
-        return KVD_ERR_CUDA;
+    } else {
+        return KVD_ERR_UNSUPPORTED_SHAPE;  // d_c 256 takes one of the two kernels above
     }
     record(g_ev_after, st);
 

@@ -79,9 +79,6 @@ struct LatentShape {
 };
 LatentShape latent_shape(int d_c);
 
-cudaError_t launch_latent_decode(int d_c, const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
-                                 const LatentArgs &a, int grid, size_t smem, cudaStream_t st);
-
 // GTA prefix attention on the latent kernel (latent_decode.cu): state = one tied group
 // (d_h 128), key = its first 64 dims + the 64-wide rope, every row sees the whole prefix.
 LatentShape tied_prefix_shape();
@@ -96,8 +93,8 @@ size_t narrow_smem_bytes();
 cudaError_t launch_gla_narrow(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid,
                               cudaStream_t st);
 
-// GLA with 65 to 128 query rows per latent head (latent_m128.cu): 64-token tiles, M = 128 MMAs,
-// q in shared memory, two softmax warps per lane quadrant; no q tensor map.
+// GLA with more than 64 query rows per latent head (latent_m128.cu), in blocks of 128 rows (one
+// CTA each): 64-token tiles, M = 128 MMAs, two softmax warps per lane quadrant; no q tensor map.
 int m128_tile_tokens();
 int m128_seg_cost();
 size_t m128_smem_bytes();

@@ -1,17 +1,17 @@
-// GLA / MLA decode (absorbed form) over a paged latent cache on 5th-generation
-// tensor cores (tcgen05, accumulators in tensor memory).
+// Latent-style attention over a paged cache on 5th-generation tensor cores (tcgen05,
+// accumulators in tensor memory), for one state shared by 128-row blocks of query rows with a
+// 64-token tile and q's rows loaded by TMA.  It serves the batched shared-prefix pass of GTA
+// (kvd_gta_prefix_decode): the state is one tied group (d_h 128), the key its first 64 dims plus
+// the 64-wide rope slice, and all B x L rows of a KV group's heads attend the prefix once,
+// without the causal mask.  (GLA decode itself runs on gla_narrow_kernel, at most 64 rows per
+// latent head, and gla_m128_kernel, more rows; MLA on the CTA-pair kernel.)
 //
-// "Hardware-Efficient Attention for Fast Decoding", section 3.3.2: h_c latent
-// heads of width d_c plus one shared RoPE key of width d_r; query head h attends
-// latent head c = h / (h_q / h_c) with key [latent_c ++ rope] and value latent_c.
-// MLA is h_c = 1, d_c = 512.  All h_q / h_c query heads of a latent head (times
-// q_len) share every loaded latent row, so the step is a real dense contraction
-// (MLA: ~2 h_q FLOPs per byte, near the B200 ridge; GLA-2: ~h_q).
+// "Hardware-Efficient Attention for Fast Decoding", section 3.3.2 gives the absorbed form this
+// follows: query head h attends state c = h / (h_q / h_c) with key [state_c ++ rope] and value
+// state_c.  The rows of a state share every loaded row, so the step is a dense contraction.
 //
-// One CTA owns one contiguous part of the (sequence, TOK-token tile) stream, one
-// latent head c and one 128-row block of the (q position, head) rows (MLA's 512 value
-// columns do not fit one CTA's tensor memory next to the scores; it runs on the CTA-pair
-// kernel instead).  Roles:
+// One CTA owns one contiguous part of the (sequence, TOK-token tile) stream, one state c and
+// one 128-row block of the (q position, head) rows.  Roles:
 //   warp 0      producer: q's rope chunk of the segment, then per tile one 3-D TMA for
 //               the latent rows and one for the rope rows (128 B swizzle), into an
 //               n-stage mbarrier ring; block-table entries a warp at a time.  Pages that
@@ -575,12 +575,6 @@ LatentShape latent_shape(int d_c) {
         s.p_bytes = 0;
     }
     return s;
-}
-
-cudaError_t launch_latent_decode(int d_c, const CUtensorMap &qm, const CUtensorMap &lm, const CUtensorMap &rm,
-                                 const LatentArgs &a, int grid, size_t smem, cudaStream_t st) {
-    if (d_c == 256) return launch_t<256, 64, 4>(qm, lm, rm, a, grid, smem, st);
-    return cudaErrorInvalidValue;
 }
 
 LatentShape tied_prefix_shape() {

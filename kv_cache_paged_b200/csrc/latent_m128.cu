@@ -1,5 +1,6 @@
-// GLA decode (absorbed form) for latent heads attended by 65 to 128 query rows: GLA-2 at
-// q_len 2 (64 heads per latent head), GLA-8 at q_len 5 to 8 (16 heads per latent head).
+// GLA decode (absorbed form) for latent heads attended by more than 64 query rows, in blocks of
+// 128 rows: GLA-2 at q_len 2 (64 heads per latent head, one block) and 4 (two blocks), GLA-8 at
+// q_len 5 to 8 (16 heads per latent head, one block) and longer speculation.
 //
 // "Hardware-Efficient Attention for Fast Decoding", section 3.3.2: h_c latent heads of width
 // d_c = 256 plus one shared RoPE key of width 64; query head h attends latent head
@@ -17,7 +18,8 @@
 // of 64 columns (P(j) written as bf16 pairs over the first 32 columns of S(j)), q's latent part
 // in [384, 512).  Shared memory: q's rope part (16 KB) and five 40 KB stages.
 //
-// One CTA owns one contiguous part of the (sequence, 64-token tile) stream and one latent head.
+// One CTA owns one contiguous part of the (sequence, 64-token tile) stream, one latent head and
+// one block of 128 rows (a latent head with more rows streams its cache once per block).
 // Roles:
 //   warps 0, 2, 3  producers: per tile the latent and rope rows of each page box by TMA (128 B
 //                  swizzle) into the ring, boxes spread over the three warps; block-table
@@ -91,9 +93,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint8_t *stage_s = smem + C::Q_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int part = blockIdx.x / a.h_c, c = blockIdx.x % a.h_c;
+    const int part = blockIdx.x / a.n_sub, sub = blockIdx.x % a.n_sub;
+    const int c = sub % a.h_c, rt = sub / a.h_c;  // latent head, block of 128 rows
     const int g = a.h_q / a.h_c;
-    const int R = g * a.L;  // 64 < R <= 128
+    const int R = g * a.L;  // > 64; this CTA's rows: [128 rt, 128 rt + 128)
     const int max_tokens = a.max_pages * a.page_size;
     const uint64_t lim_ns = a.wait_limit_ns;
 
@@ -131,13 +134,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     uint32_t m_tile = 0, m_s = 0, m_pv = 0, m_q = 0;  // MMA issuer
     uint32_t x_tile = 0, x_s = 0, x_pv = 0, x_x = 0;  // softmax (x_x: pair exchanges)
 
-    // softmax thread geometry: row n = 32 qd + lane (MMA row = TMEM lane), score half `half`
+    // softmax thread geometry: MMA row (TMEM lane) n_loc = 32 qd + lane, row n_row of the latent
+    // head, score half `half`
     const bool smx_warp = warp >= 4 && warp < 4 + NSMX;
     const int qd = warp & 3;
     const int half = smx_warp ? (warp - 4) >> 2 : 0;
-    const int n_row = smx_warp ? 32 * qd + lane : 0;
+    const int n_loc = smx_warp ? 32 * qd + lane : 0;
+    const int n_row = 128 * rt + n_loc;
     const bool row_ok = smx_warp && n_row < R;
-    const bool warp_live = 32 * qd < R;  // some row of this quadrant is real
+    const bool warp_live = 128 * rt + 32 * qd < R;  // some row of this quadrant is real
     const int i_row = row_ok ? n_row / g : 0;
     const int head = row_ok ? c * g + n_row % g : 0;
     const uint32_t s_lanes = (uint32_t)(qd * 32) << 16;
@@ -152,7 +157,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t dst = smem_u32(q_s);
 #pragma unroll
             for (int u = 4 * half; u < 4 * half + 4; ++u)
-                cp_async16(dst + sw128((uint32_t)n_row, (uint32_t)u), src + C::DC + u * 8, q_pol);
+                cp_async16(dst + sw128((uint32_t)n_loc, (uint32_t)u), src + C::DC + u * 8, q_pol);
         }
         cp_async_arrive(&qfull_bar);
         const uint4 *lat = (const uint4 *)(src + half * (C::DC / 2));
@@ -182,15 +187,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // before what the other writes after it (P over those columns).
     auto exchange = [&](float v0, float v1, float &p0, float &p1) -> bool {
         const uint32_t bf = x_x & 1;
-        xch_sh[bf][half][n_row][0] = v0;
-        xch_sh[bf][half][n_row][1] = v1;
+        xch_sh[bf][half][n_loc][0] = v0;
+        xch_sh[bf][half][n_loc][1] = v1;
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&xbar[qd][bf]);
         if (!mbar_wait_warp(&xbar[qd][bf], (x_x >> 1) & 1, &abort_sh, a.err, lim_ns)) return false;
         tc_fence_after();
-        p0 = xch_sh[bf][half ^ 1][n_row][0];
-        p1 = xch_sh[bf][half ^ 1][n_row][1];
+        p0 = xch_sh[bf][half ^ 1][n_loc][0];
+        p1 = xch_sh[bf][half ^ 1][n_loc][1];
         ++x_x;
         return true;
     };
@@ -279,10 +284,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     return raw * a.page_size + (t * TOK + kbox * box_tok) % a.page_size;
                 };
-                // warp 0 of the first latent head's CTA brings the pages of tile t + PF into L2
-                // when it loads tile t (whole pages, every latent head and the rope rows, one
-                // untiled bulk prefetch each)
-                const bool pf_warp = warp == 0 && c == 0;
+                // warp 0 of the part's first CTA (first latent head and row block) brings the pages
+                // of tile t + PF into L2 when it loads tile t (whole pages, every latent head and
+                // the rope rows, one untiled bulk prefetch each)
+                const bool pf_warp = warp == 0 && sub == 0;
                 const size_t lat_page = (size_t)a.page_size * a.h_c * C::DC * 2, rope_page = (size_t)a.page_size * 128;
                 int pf_next_page = -1;  // logical page index prefetched next (pages already done: below)
                 auto raw_page = [&](int t) -> int {  // lane j: the j-th page of tile t

@@ -241,9 +241,10 @@ def test_latent_page_permutation_bit_identical(cuda_device):
     assert torch.equal(lse1, lse2)
 
 
-# ----------------------------------------------------------------------------- 65 to 128 rows per latent head
-# GLA-2 at q_len 2 and GLA-8 at q_len 5 to 8 run on the 128-row kernel (64-token tiles, M = 128,
-# two softmax warps per lane quadrant that exchange their row maxima every tile).
+# ----------------------------------------------------------------------------- more than 64 rows per latent head
+# GLA-2 from q_len 2 and GLA-8 from q_len 5 run on the 128-row kernel (64-token tiles, M = 128,
+# two softmax warps per lane quadrant that exchange their row maxima every tile; one CTA per
+# block of 128 rows).
 @pytest.mark.parametrize("num_parts", [1, 3, 50, 148])
 def test_m128_forced_splits(cuda_device, num_parts):
     inp = small(2, 256, B=5, L=2, seqlens=("uniform", 16, 1500), seed=311 + num_parts)
@@ -271,6 +272,14 @@ def test_m128_row_counts(cuda_device, h_c, h_q, L):
     """R = 80, 128, 96 and 128 rows: the last lane quadrants partly or wholly without rows."""
     inp = small(h_c, 256, h_q=h_q, L=L, seqlens=("uniform", L + 8, 500), seed=337 + h_c + L)
     check(inp, num_parts=3, what=f"h_c={h_c} h_q={h_q} L={L}")
+
+
+@pytest.mark.parametrize("L,parts", [(3, 0), (4, 7), (6, 3)])
+def test_m128_row_blocks(cuda_device, L, parts):
+    """More than 128 rows per latent head: GLA-2 at q_len 3, 4 and 6 (192, 256 and 384 rows) runs
+    one CTA per 128-row block, the last block partly without rows at q_len 3."""
+    inp = small(2, 256, L=L, B=4, seqlens=("uniform", L + 16, 900), seed=359 + L)
+    check(inp, num_parts=parts, what=f"GLA-2 L={L} parts={parts}")
 
 
 def test_m128_peaky_softmax(cuda_device):

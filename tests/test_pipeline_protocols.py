@@ -1,7 +1,7 @@
 """Barrier protocols of the decode kernels, modelled on the CPU.
 
 Every warp role of the GQA/GTA kernel (group_decode.cu: box loads or gathered tiles), of the
-GLA kernels (latent_decode.cu, latent_narrow.cu, latent_m128.cu) and of the MLA CTA-pair kernel
+latent kernels (latent_decode.cu: the GTA shared-prefix pass; latent_narrow.cu and latent_m128.cu: GLA) and of the MLA CTA-pair kernel
 (latent_pair.cu) is a coroutine that waits on and arrives at its mbarriers in the order the
 kernel does; TMA copies, bulk copies to the peer CTA and tcgen05.commit arrivals complete later,
 in random order.  Random schedules over several segment patterns and stage counts must all
