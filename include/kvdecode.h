@@ -125,8 +125,10 @@ typedef struct {
 
 /*
  * GLA / MLA (absorbed).  d_c in {256, 512}, d_r == 64, h_q % h_c == 0, h_q / h_c divides or is
- * a multiple of 128, (h_q / h_c) * L <= 8192; any page_size >= 1 (multiples of 64 load
- * whole tiles, other sizes are gathered token by token).
+ * a multiple of 128, (h_q / h_c) * L <= 8192; any page_size >= 1.  GLA (d_c 256) loads a
+ * tile (96 tokens with at most 64 query rows per latent head, 64 with more) in boxes of
+ * gcd(tile, page_size) tokens when that is at least 16, MLA whole 64-token tiles when
+ * page_size is a multiple of 64; other page sizes are gathered token by token.
  */
 typedef struct {
     const void *q;            /* bf16 [B, L, h_q, d_c + d_r] = [latent ++ rope] */
@@ -217,9 +219,9 @@ int kvd_merge_states(const void *out_a, const float *lse_a, const void *out_b, c
  * segments[c * cap * 6 ...] and the record count at counts[c] (device
  * pointers).  A count above `cap` means records were dropped.  seg_cost >= 0:
  * each non-empty sequence counts as seg_cost extra tiles placed before its
- * own when the stream is cut into parts of equal size (the GLA kernel for at
- * most 64 rows per latent head plans with 3, GTA with 128 / tile, the others
- * with 0).
+ * own when the stream is cut into parts of equal size (the GLA kernels plan
+ * with 3 for at most 64 rows per latent head and 4 for more, GTA with
+ * 128 / tile, the others with 0).
  */
 int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t seg_cost, int32_t max_tokens,
              int32_t num_parts, int32_t *segments, int32_t *counts, int32_t cap, kvd_stream_t stream);
