@@ -220,7 +220,7 @@ int kvd_merge_states(const void *out_a, const float *lse_a, const void *out_b, c
  * pointers).  A count above `cap` means records were dropped.  seg_cost >= 0:
  * each non-empty sequence counts as seg_cost extra tiles placed before its
  * own when the stream is cut into parts of equal size (the GLA kernels plan
- * with 3 for at most 64 rows per latent head and 4 for more, GTA with
+ * with 3 for at most 64 rows per latent head and 7 for more, GTA with
  * 128 / tile, the others with 0).
  */
 int kvd_plan(const int32_t *seqlens, int32_t B, int32_t tile, int32_t seg_cost, int32_t max_tokens,

@@ -607,8 +607,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 int m128_tile_tokens() { return M128_TOK; }
 // A segment start costs the CTA a few µs (its q rows, the ring refilling, the epilogue of the
-// segment before it) against ~1 µs per 64-token tile at the HBM rate.
-int m128_seg_cost() { return 4; }
+// segment before it) against ~1.4 µs per 64-token tile; measured on GLA-2 at q_len 2 (step µs):
+// 613.4 with 2, 605.2 with 4, 596.8 with 7.
+int m128_seg_cost() { return 7; }
 size_t m128_smem_bytes() { return M128Cfg::SMEM; }
 
 cudaError_t launch_gla_m128(const CUtensorMap &lm, const CUtensorMap &rm, const LatentArgs &a, int grid,
