@@ -1,4 +1,4 @@
-"""GQA / GTA decode on the GPU against the fp64 oracle (the benchmark spec tolerance), plus
+"""GQA / GTA decode on the GPU against the fp64 oracle (the stated output tolerance), plus
 bit-exact indexing, split invariance and device error reporting."""
 import numpy as np
 import pytest

@@ -1,4 +1,4 @@
-"""GLA / MLA (absorbed) decode on the GPU against the fp64 oracle (the benchmark spec tolerance)."""
+"""GLA / MLA (absorbed) decode on the GPU against the fp64 oracle (the stated output tolerance)."""
 import numpy as np
 import pytest
 
