@@ -272,7 +272,7 @@ def test_model_detects_a_missing_arrival():
     assert short(0, (3,), 2) == "stuck"
 
 
-def q_in_cta_model(seed, segs, nstage, pair, skip_exchange=False):
+def q_in_cta_model(seed, segs, nstage, pair, skip_exchange=False, log=None, no_exchange=False):
     """gla_narrow_kernel (pair=False: four softmax warps) and gla_m128_kernel (pair=True: eight,
     two per TMEM lane quadrant).  The softmax warps write each segment's q themselves: for the
     first segment at its start, for every later one as soon as the previous segment's last score
@@ -280,7 +280,9 @@ def q_in_cta_model(seed, segs, nstage, pair, skip_exchange=False):
     once its tensor-memory writes are out.  The MMA warp waits for q before a segment's first
     score product.  With `pair` the two warps of a quadrant exchange their row maxima every tile
     and their row sums at each segment end through two mbarriers of two arrivals, used
-    alternately."""
+    alternately.  With `log`, every softmax warp appends ("read", quadrant, half, tile) when it
+    has loaded its scores and ("write", quadrant, half, tile) when it stores P over the S
+    buffer."""
     rnd = random.Random(seed)
     events = []
     nsmx = 8 if pair else 4
@@ -330,7 +332,7 @@ def q_in_cta_model(seed, segs, nstage, pair, skip_exchange=False):
                 c["qfull"].arrive()  # the warp's tensor-memory writes are out
 
         def exchange():
-            if skip_exchange and w == 4 and xx[0] == 1:
+            if no_exchange or (skip_exchange and w == 4 and xx[0] == 1):
                 return
             b = xx[0] % 2
             xbar[q][b].arrive()
@@ -344,10 +346,15 @@ def q_in_cta_model(seed, segs, nstage, pair, skip_exchange=False):
                 yield from wait(lambda: c["sfull"][x % 2].ready(x // 2))
                 if j == n - 1 and si + 1 < len(segs):
                     load_q()
+                if log is not None:
+                    log.append(("read", q, w // 4, x))
+                    yield
                 if pair:
                     yield from exchange() or ()
                 if x > 0 and rnd.random() < 0.3:  # lazy rescale: O settled after P.V(x - 1)
                     yield from wait(lambda: c["empty"][(x - 1) % nstage].ready((x - 1) // nstage))
+                if log is not None:
+                    log.append(("write", q, w // 4, x))
                 c["pfull"][x % 2].arrive()
                 x += 1
             yield from wait(lambda: c["empty"][(x - 1) % nstage].ready((x - 1) // nstage))  # epilogue
@@ -366,6 +373,29 @@ def test_q_in_cta_protocols_finish_without_parity_aliasing(pair, segs, nstage):
     for seed in range(25):
         assert q_in_cta_model(seed, segs, nstage, pair) == "ok", seed
     assert not ALIAS, ALIAS[:5]
+
+
+def test_m128_p_over_s_follows_the_partners_score_read():
+    """In the 128-row kernel the warp of a pair that holds the last 32 scores of a row writes its
+    P over S columns [16, 32), which hold scores of the other warp's half: the exchange has to
+    order the other warp's read of tile x before this write, in every schedule."""
+    for seed in range(40):
+        log = []
+        assert q_in_cta_model(seed, (3, 1, 4), 3, True, log=log) == "ok", seed
+        pos = {e: i for i, e in enumerate(log)}
+        for (kind, q, h, x), i in pos.items():
+            if kind == "write":
+                assert pos[("read", q, 1 - h, x)] < i, (seed, q, h, x)
+
+
+def test_m128_ordering_check_bites_without_the_exchange():
+    """Without the exchange some schedule lets a warp write its P before its partner read."""
+    def violated(seed):
+        log = []
+        assert q_in_cta_model(seed, (3, 1, 4), 3, True, log=log, no_exchange=True) == "ok"
+        pos = {e: i for i, e in enumerate(log)}
+        return any(kind == "write" and pos[("read", q, 1 - h, x)] > i for (kind, q, h, x), i in pos.items())
+    assert any(violated(seed) for seed in range(40))
 
 
 def test_pair_exchange_model_detects_a_skipped_exchange():
