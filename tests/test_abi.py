@@ -223,6 +223,17 @@ def test_gla_any_page_size_is_accepted(lib, S, d_c, h_c):
     assert lib.kvd_gla_workspace_size(ctypes.byref(_gla_params(page_size=S, d_c=d_c, h_c=h_c))) > 0
 
 
+@pytest.mark.parametrize("L,S", [(1, 1), (1, 16), (2, 1), (2, 48), (4, 64), (6, 8)])
+def test_gla2_every_row_count_and_page_size_is_planned(lib, L, S):
+    """GLA-2 at 64, 128, 256 and 384 rows per latent head (the narrow kernel, the 128-row kernel
+    in one or several row blocks), with boxed and gathered page sizes: the workspace holds the
+    split partials of every row."""
+    p = _gla_params(L=L, page_size=S)
+    slots, rows = 2 + 4 - 1, L * 128
+    assert lib.kvd_gla_workspace_size(ctypes.byref(p)) == (
+        256 + ((slots * rows * 4 + 255) // 256) * 256 + slots * rows * 256 * 4)
+
+
 def test_gla_workspace_size(lib):
     p = _gla_params(L=2, d_c=512, h_c=1, page_size=64)
     n = lib.kvd_gla_workspace_size(ctypes.byref(p))
