@@ -635,7 +635,9 @@ def main():
     e2e_mode = "cuda graph of the steps, one replay timed"
     try:
         graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=origin):
+        # thread-local capture: CUDA calls of other threads (NCCL's watchdog under torchrun) do not
+        # invalidate it
+        with torch.cuda.graph(graph, stream=origin, capture_error_mode="thread_local"):
             enqueue_loop(origin)
         with torch.cuda.stream(origin):
             graph.replay()              # warm
