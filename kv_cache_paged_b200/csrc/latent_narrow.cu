@@ -18,10 +18,11 @@
 //
 // One CTA owns one contiguous part of the (sequence, TOK-token tile) stream and one latent
 // head.  Roles:
-//   warp 0      producer: per tile the latent and rope rows of each page box by TMA (128 B
-//               swizzle) into an NSTAGE ring; block-table entries one lane per box.  Pages
-//               that are not whole boxes are gathered token by token with cp.async by warps
-//               0, 2 and 3.
+//   warps 0,2,3 producers: per tile the latent and rope rows of each page box by TMA (128 B
+//               swizzle) into an NSTAGE ring, boxes spread over the three warps; block-table
+//               entries one lane per box.  Pages that are not whole boxes are gathered token by
+//               token with cp.async by five warps (0, 2, 3, 8, 9: the gather instantiation of
+//               the kernel has 320 threads).
 //   warp 1      MMA issuer (one thread).
 //   warps 4..7  softmax, two threads per row (lanes l and l + 16 of the quadrant's warp take
 //               the first and second half of the row's TOK scores through the half-warp
